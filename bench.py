@@ -1,0 +1,400 @@
+"""Benchmark of the block-sparse / piecewise attention hot path on B200.
+
+One step = one pass of the whole PISA path over one batch of the workload:
+bsa_precompute -> bsa_route -> bsa_forward (the fixed-mask builder is built once per
+model and is not part of a PISA step). Default workload: video PISA, batch 1, 40 heads,
+L = 16384 (16 frames x 32 x 32), d = 128, block 128, density 12.5% (top-16 of 128).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu]
+
+Prints ONE JSON line on rank 0. With torchrun (N > 1) every rank runs the same
+workload on its own GPU (replicas, weak scaling; the path needs no data exchange) and
+the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from piecewise_attention_diffusion_b200 import synth  # noqa: E402
+
+METRIC = "bsa_forward effective TFLOPS (executed FLOPs) over precompute+route+forward"
+LAMBDA = 1.0
+
+
+# ------------------------------------------------------------------ FLOP counting
+def forward_flops(w, k_top: int, mode: str) -> float:
+    """Executed FLOPs of bsa_forward: per (batch, head, query block)
+    k * 4 B^2 d  (+ PISA: B * (4 d |U_i| + 2 d^2)); exps and softmax not counted."""
+    M, B, d = w.n_blocks, w.block, w.head_dim
+    per_qb = k_top * 4.0 * B * B * d
+    if mode == "pisa":
+        per_qb += B * (4.0 * d * (M - k_top) + 2.0 * d * d)
+    return w.batch * w.heads * M * per_qb
+
+
+def precompute_flops(w) -> float:
+    """K_j^T V_j per block (2 B d^2), counted once."""
+    return w.batch * w.heads * w.n_blocks * 2.0 * w.block * w.head_dim ** 2
+
+
+def route_flops(w) -> float:
+    """pooled-query x centroid scores (2 M^2 d per head)."""
+    return w.batch * w.heads * 2.0 * w.n_blocks ** 2 * w.head_dim
+
+
+def forward_bytes(w, mode: str) -> float:
+    """Algorithmic HBM bytes of bsa_forward: Q, K, V read and O written once (bf16),
+    plus the fp32 statistics for PISA."""
+    BH, L, d, M = w.batch * w.heads, w.seq_len, w.head_dim, w.n_blocks
+    b = 4.0 * BH * L * d * 2
+    if mode == "pisa":
+        b += BH * (2 * M * d + d * d) * 4
+    return b
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                p = [x.strip() for x in ln.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
+                                                         if r[3].replace(".", "").isdigit())}
+
+
+# ------------------------------------------------------------------ dist helpers
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d["bf16_tflops"], "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def load_traffic(w) -> float | None:
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary of
+    the current kernel (None when no capture matches the current kernel)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(w.name)
+    return None if e is None else e.get("bytes_per_launch")
+
+
+# -------------------------------------------------------------- CPU oracle timing
+def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
+    """Time the fp64 oracle (as it stands) on `heads_sample` full heads and scale to
+    the whole workload by the head count."""
+    import oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    heads = list(range(heads_sample))
+    q, k, v = synth.make_qkv(w, seed=seed, heads=heads)
+    scale = 1 / math.sqrt(w.head_dim)
+    t0 = time.perf_counter()
+    for h in heads:
+        qf, kf, vf = (x[h].to(torch.float64).numpy() for x in (q, k, v))
+        kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block)
+        rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale)
+        if w.mode == "pisa":
+            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar)
+        else:
+            orc.keep_or_drop_head(qf, kf, vf, rp, ci, w.block, scale)
+    dt = time.perf_counter() - t0
+    BH = w.batch * w.heads
+    return {"seconds_sample": dt, "seconds_full_est": dt * BH / len(heads), "cores": threads,
+            "sample": f"{len(heads)} of {BH} heads, each fully precomputed, routed and "
+                      f"attended (all {w.n_blocks} query blocks); time scaled by heads"}
+
+
+# --------------------------------------------------------------------- our arm
+def run_ours(args, w, world, rank, local):
+    from piecewise_attention_diffusion_b200 import bsattn as b
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    k_top = w.top_k()
+    BH, M, L, d = w.batch * w.heads, w.n_blocks, w.seq_len, w.head_dim
+    q, k, v = synth.make_qkv(w, seed=args.seed + rank)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    stats = dict(kbar=torch.empty(BH, M, d, **f32), vsum=torch.empty(BH, M, d, **f32),
+                 Hbar=torch.empty(BH, d, d, **f32), Mnorm=torch.empty(BH, M, **f32))
+    rp = torch.empty(BH * (M + 1), dtype=torch.int32, device=dev)
+    ci = torch.empty(BH * M * k_top, dtype=torch.int32, device=dev)
+    O = torch.empty_like(qd)
+    ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
+    ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
+    mode = b.MODE_PISA if w.mode == "pisa" else b.MODE_KEEP_OR_DROP
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qx, kx, vx, ev=None):
+        if ev:
+            ev[0].record(stream)
+        b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
+                         stats["Mnorm"], None, ws_p, st)
+        if ev:
+            ev[1].record(stream)
+        b.bsa_route(qx, stats["kbar"], stats["Mnorm"], w.block, k_top, LAMBDA, 0.0, rp, ci,
+                    None, st)
+        if ev:
+            ev[2].record(stream)
+        b.bsa_forward(qx, kx, vx, w.block, rp, ci, 1, mode, stats["kbar"], stats["vsum"],
+                      stats["Hbar"], 0.0, O, None, ws_f, st)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step(qd, kd, vd)
+    torch.cuda.synchronize()
+    if st.item() != 0:
+        raise RuntimeError(f"device status {b.status_string(st.item())}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(qd, kd, vd, evs[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = clk.summary()
+    ms_total = t_start.elapsed_time(t_end)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    route_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    fwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    ms_step = max_over_ranks(ms_total / args.steps, world)
+    fwd_ms = max_over_ranks(fwd_ms, world)
+    if st.item() != 0:
+        raise RuntimeError(f"device status {b.status_string(st.item())}")
+
+    F_fwd = forward_flops(w, k_top, w.mode)
+    F_step = F_fwd + precompute_flops(w) + route_flops(w)
+    value = world * F_step / (ms_step * 1e-3) / 1e12
+    pk = peaks()
+    achieved = F_fwd / (fwd_ms * 1e-3) / 1e12
+
+    # ---- end to end: host (pinned) inputs -> device -> path -> host output
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        Oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            step(qd, kd, vd)
+            Oh.copy_(O, non_blocking=True)
+        torch.cuda.synchronize()
+        e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e_s.record(stream)
+        for _ in range(args.steps):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            step(qd, kd, vd)
+            Oh.copy_(O, non_blocking=True)
+        e_e.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world)
+        e2e = {"value": round(world * F_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": int(3 * q.numel() * 2),
+               "d2h_bytes_per_step": int(O.numel() * 2)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: Q ~ N(0,1); K, V = smooth 3-D field + 0.3 N(0,1))",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": L,
+                   "head_dim": d, "block": w.block, "mode": w.mode, "density": w.density,
+                   "k_top": k_top, "lambda": LAMBDA, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 (Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB)"},
+        "forward_ms": round(fwd_ms, 4), "forward_tflops": round(achieved, 3),
+        "precompute_ms": round(pre_ms, 4), "route_ms": round(route_ms, 4),
+        "forward_gflop": round(F_fwd / 1e9, 3),
+        "dense_equiv_tflops": round(4.0 * BH * L * L * d / (fwd_ms * 1e-3) / 1e12, 3),
+        "roofline": {"kernel": "bsa_forward", "bound": "tensor", "achieved": round(achieved, 3),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "peak_source": f"{pk['source']} bf16_tflops (burst)",
+                     "traffic": load_traffic(w),
+                     "algorithmic_bytes": forward_bytes(w, w.mode)},
+        "clocks": clocks,
+        "gpu_launches": 6 * args.steps,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cs = oracle_sample(w, k_top, args.cpu_heads, args.seed)
+        line["cpu_baseline"] = {"value": round(F_step / cs["seconds_full_est"] / 1e12, 6),
+                                "unit": "TFLOP/s", "cores": cs["cores"], "kind": "oracle",
+                                "sample": cs["sample"],
+                                "seconds_full_est": round(cs["seconds_full_est"], 2)}
+    return line
+
+
+# --------------------------------------------------------------- reference arm
+def run_reference(args, w, world, rank):
+    """The fp64 oracle, as it stands, on the host cores: each step a bounded sample."""
+    k_top = w.top_k()
+    F_step = forward_flops(w, k_top, w.mode) + precompute_flops(w) + route_flops(w)
+    for _ in range(args.warmup):
+        oracle_sample(w, k_top, 1, args.seed)
+    times, info = [], None
+    for _ in range(args.steps):
+        info = oracle_sample(w, k_top, args.ref_heads, args.seed)
+        times.append(info["seconds_full_est"])
+    sec = float(np.mean(times))
+    value = F_step / sec / 1e12
+    cpu = {"value": round(value, 6), "unit": "TFLOP/s", "cores": info["cores"], "kind": "oracle",
+           "sample": info["sample"]}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (same generator and seed)",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads,
+                       "seq_len": w.seq_len, "head_dim": w.head_dim, "block": w.block,
+                       "mode": w.mode, "density": w.density, "k_top": k_top,
+                       "lambda": LAMBDA, "parallelism": "host cores"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="video_pisa")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--ref-heads", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = synth.workloads()[args.workload]
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, w, world, rank)), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    try:
+        line = run_ours(args, w, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

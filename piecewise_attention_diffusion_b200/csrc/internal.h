@@ -1,0 +1,50 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bsattn.h"
+
+namespace bsa {
+
+struct Shape {
+  int Bt, H, L, d, block;
+  int BH() const { return Bt * H; }
+  int M() const { return L / block; }
+};
+
+// Workspace size of each call (bytes); 0 if none.
+size_t precompute_workspace(const Shape& s);
+size_t forward_workspace(const Shape& s);
+
+cudaError_t launch_build_mask(const bsa_mask_desc& desc, int M, int32_t* row_ptr,
+                              int32_t* col_idx, int64_t cap, int32_t* status,
+                              cudaStream_t st);
+
+cudaError_t launch_precompute(const Shape& s, const void* K, const void* V, float* kbar,
+                              float* vsum, float* Hbar, float* Mnorm, float* Hblk,
+                              void* ws, int32_t* status, cudaStream_t st);
+
+cudaError_t launch_route(const Shape& s, const void* Q, const float* kbar,
+                         const float* Mnorm, int k_top, float lambda, float scale,
+                         int32_t* row_ptr, int32_t* col_idx, float* scores,
+                         int32_t* status, cudaStream_t st);
+
+struct ForwardArgs {
+  Shape s;
+  const void *Q, *K, *V;
+  const int32_t *row_ptr, *col_idx;
+  int64_t nnz_total;
+  int csr_per_head;
+  int mode;
+  const float *kbar, *vsum, *Hbar;
+  float scale;
+  void* O;
+  float* lse;
+  void* ws;
+  int32_t* status;
+};
+
+cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t st);
+
+}  // namespace bsa
