@@ -68,31 +68,36 @@ def forward_bytes(w, mode: str) -> float:
 
 # ---------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 50 ms, timestamped) of SM clock and throttle reasons;
+    summary() keeps the samples that fall inside the timed region (widened by 0.25 s
+    on both sides so that a short region still gets samples taken under load)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.3)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -101,25 +106,33 @@ class ClockSampler:
             self.f.close()
 
     def summary(self) -> dict:
+        import datetime
         if self.proc is None or self.path is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
         with open(self.path) as f:
             for ln in f:
                 p = [x.strip() for x in ln.split(",")]
-                if len(p) >= 9 and p[1].replace(".", "").isdigit():
-                    rows.append(p)
+                if len(p) < 10 or not p[2].replace(".", "").isdigit():
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                rows.append([ts] + p[1:])
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
-        mx = max(float(r[2]) for r in rows)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        loaded = [s for s in sm if s > 0.5 * mx] or sm
-        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
-                                                         if r[3].replace(".", "").isdigit())}
+        inside = [r for r in rows if self.t0 - 0.25 <= r[0] <= self.t1 + 0.25]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": [f"no samples in the timed region ({len(rows)} outside)"]}
+        sm = [float(r[2]) for r in inside]
+        mx = max(float(r[3]) for r in inside)
+        reasons = sorted({self.REASONS[i] for r in inside for i in range(4)
+                          if r[6 + i] == "Active"})
+        pw = [float(r[4]) for r in inside if r[4].replace(".", "").isdigit()]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(inside), "power_w_max": max(pw) if pw else None,
+                "window_s": round(self.t1 - self.t0, 3)}
 
 
 # ------------------------------------------------------------------ dist helpers
@@ -236,6 +249,8 @@ def run_ours(args, w, world, rank, local):
         if ev:
             ev[3].record(stream)
 
+    clk = ClockSampler(local).start()
+    time.sleep(0.5)  # let nvidia-smi start sampling before the GPU work begins
     for _ in range(args.warmup):
         step(qd, kd, vd)
     torch.cuda.synchronize()
@@ -244,16 +259,16 @@ def run_ours(args, w, world, rank, local):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        t_start.record(stream)
-        for s in range(args.steps):
-            step(qd, kd, vd, evs[s])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-    clocks = clk.summary()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk.t0 = time.time()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(qd, kd, vd, evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk.t1 = time.time()
+    barrier(world)
     ms_total = t_start.elapsed_time(t_end)
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     route_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
@@ -300,6 +315,8 @@ def run_ours(args, w, world, rank, local):
                "h2d_bytes_per_step": int(3 * q.numel() * 2),
                "d2h_bytes_per_step": int(O.numel() * 2)}
 
+    clk.stop()
+    clocks = clk.summary()
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -364,10 +381,12 @@ def run_reference(args, w, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="video_pisa")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller profiling captures)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-heads", type=int, default=8)
     ap.add_argument("--ref-heads", type=int, default=2)
@@ -377,6 +396,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = synth.workloads()[args.workload]
+    if args.heads > 0:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
 
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -47,4 +47,9 @@ struct ForwardArgs {
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t st);
 
+// Tensor-core attention kernel (forward_tc.cu); `flag` is the validation result, the
+// first word of the forward workspace.
+size_t forward_tc_workspace(const Shape& s);
+cudaError_t launch_forward_tc(const ForwardArgs& a, const int32_t* flag, cudaStream_t st);
+
 }  // namespace bsa

@@ -165,7 +165,18 @@ def _forward_check(w, q, k, v, rp, ci, per_head, mode, stats_np, qblocks=None, h
             got_l = f64(lg[h, rows])
             fin = np.isfinite(wl)
             assert (np.isneginf(got_l) == ~fin).all()
-            np.testing.assert_allclose(got_l[fin], wl[fin], atol=2e-3, rtol=1e-4)
+            tol = np.full(len(rows), 2e-3)
+            if mode == b.MODE_PISA:
+                # The centroid sweep runs on the tensor cores with kbar rounded to bf16
+                # (unit roundoff 2^-8): each centroid score moves by at most
+                # s * sum_c |q_c| |kbar_c| 2^-8, and the log-denominator by at most the
+                # largest such shift.
+                kbar = stats_np[0][h]
+                shift = scale * np.abs(qf[h][rows]) @ np.abs(kbar).T * 2.0 ** -8
+                tol += shift.max(axis=1)
+            err = np.abs(got_l[fin] - wl[fin])
+            assert (err <= tol[fin]).all(), float((err - tol[fin]).max())
+    print(f"[parity] {w.name} mode={mode} max-abs {worst[0]:.2e} rel-L2 {worst[1]:.2e}")
     return worst
 
 
@@ -314,5 +325,6 @@ def test_pipeline_full_size_sampled(name, heads, qblocks):
     for h in heads:
         blocks = list(range(M)) if qblocks is None else qblocks
         rows = np.concatenate([np.arange(i * w.block, (i + 1) * w.block) for i in blocks])
-        assert_close_out(Og[h, rows], ref[h][0], f"{name} head {h}")
+        mx, rl = assert_close_out(Og[h, rows], ref[h][0], f"{name} head {h}")
+        print(f"[parity] {name} head {h} max-abs {mx:.2e} rel-L2 {rl:.2e}")
     assert torch.isfinite(O.float()).all()
