@@ -130,7 +130,6 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ[2] = {smem, smem + C::QBYTES};
   unsigned char* sSlot = smem + 2 * C::QBYTES;
   __shared__ Barriers bars;
   __shared__ uint32_t tmem_base_sh;
@@ -211,7 +210,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_arrive_expect_tx(&bars.q_full[qb], p.qbox * D * 2);
 #pragma unroll
         for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(sQ[qb] + h * kBQ * 128, &tmQ, &bars.q_full[qb], h * 64, qt * kBQ, bh);
+          tma_load_3d(smem + qb * C::QBYTES + h * kBQ * 128, &tmQ, &bars.q_full[qb], h * 64, qt * kBQ, bh);
         ++q_issued;
         Lists lk = lists, lv = lists;
         for (int t = 0; t < n && ok; ++t) {
@@ -272,7 +271,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int qb = it & 1;
         if (!mbar_wait(&bars.q_full[qb], (it >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ[qb]);
+        const uint32_t q_addr = smem_u32(smem + qb * C::QBYTES);
         bool o_free_done = (it == 0);
         auto wait_o_free = [&]() -> bool {
           if (o_free_done) return true;
@@ -392,7 +391,8 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           }
           tmem_wait_ld();
         }
-        const int N = chunk ? kChunk : BKV;
+        // tile width: 128 for centroid chunks, BKV for exact tiles (compile-time for 128)
+        const int N = BKV == kChunk ? kChunk : (chunk ? kChunk : BKV);
         if (!chunk) {
           if (C::QBPT == 2) {
             const int j = lists.next();
@@ -418,18 +418,20 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           for (int x = 0; x < kChunk; ++x)
             if (x >= valid || ((excl[x >> 5] >> (x & 31)) & 1u)) s[x] = -INFINITY;
         }
-        // row max (log2 domain)
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max (log2 domain); 8 independent chains keep the FMNMX latency hidden
+        float mxa[8];
 #pragma unroll
-        for (int x = 4; x < 128; x += 4) {
+        for (int a = 0; a < 8; ++a) mxa[a] = s[a];
+#pragma unroll
+        for (int x = 8; x < 128; x += 8) {
           if (x < N) {
-            mx0 = fmaxf(mx0, s[x]);
-            mx1 = fmaxf(mx1, s[x + 1]);
-            mx2 = fmaxf(mx2, s[x + 2]);
-            mx3 = fmaxf(mx3, s[x + 3]);
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mxa[a] = fmaxf(mxa[a], s[x + a]);
           }
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+        const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                               fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
+                         p.scale_log2;
         const bool need = mx > m_run + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mx : m_run;
@@ -456,31 +458,31 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           m_run = m_new;
         }
         const float m_ref = m_run == -INFINITY ? 0.f : m_run;
-        float sum0 = 0.f, sum1 = 0.f;
-        uint32_t pk[64];
+        // P = 2^(s*scale_log2 - m) as bf16 pairs, written back over the first N/2
+        // columns of this S buffer one 64-column half at a time (all S values are
+        // already in registers, so the overwrite is safe)
+        const uint32_t p_addr = tmem + lane_addr + (buf ? 128u : 0u);
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int x = 0; x < 128; x += 2) {
-          if (x < N) {
-            const float e0 = ex2(fmaf(s[x], p.scale_log2, -m_ref));
-            const float e1 = ex2(fmaf(s[x + 1], p.scale_log2, -m_ref));
-            sum0 += e0;
-            sum1 += e1;
-            pk[x / 2] = pack_bf16x2(e0, e1);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (hf * 64 < N) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int x = 0; x < 64; x += 2) {
+              const float e0 = ex2(fmaf(s[hf * 64 + x], p.scale_log2, -m_ref));
+              const float e1 = ex2(fmaf(s[hf * 64 + x + 1], p.scale_log2, -m_ref));
+              sm[(x / 2) & 7] += e0 + e1;
+              pk[x / 2] = pack_bf16x2(e0, e1);
+            }
+            tmem_st32(p_addr + hf * 32, pk);
           }
         }
-        const float rs = sum0 + sum1;
+        const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
         if (chunk) {
           l += (float)BKV * rs;
           sa += rs;
         } else {
           l += rs;
-        }
-        const uint32_t p_addr = tmem + lane_addr + (buf ? 128u : 0u);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (c * 64 < N) {
-            tmem_st32(p_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + c * 32));
-          }
         }
         tmem_wait_st();
         tc_fence_before();
