@@ -56,8 +56,13 @@ typedef enum {
   BSA_ERR_BAD_CSR = 4,       /* block lists malformed (device-detected)              */
   BSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (device-detected) */
   BSA_ERR_WORKSPACE = 6,     /* workspace null or smaller than bsa_workspace_bytes   */
-  BSA_ERR_CAPACITY = 7       /* an output list would exceed its capacity (device)    */
+  BSA_ERR_CAPACITY = 7,      /* an output list would exceed its capacity (device)    */
+  BSA_ERR_SCRATCH_LIMIT = 8  /* bsa_forward_noalloc: the shape needs more scratch than
+                                BSA_NOALLOC_SCRATCH_BYTES                            */
 } bsa_status;
+
+/* Size of the device scratch array built into the library for bsa_forward_noalloc. */
+#define BSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 typedef enum {
   BSA_MODE_KEEP_OR_DROP = 0, /* [BSA] §3.3: softmax over the selected blocks only      */
@@ -179,6 +184,32 @@ BSA_API bsa_status bsa_forward(const void* Q, const void* K, const void* V, int3
                        int32_t mode, const float* kbar, const float* vsum,
                        const float* Hbar, float scale, void* O, float* lse,
                        void* workspace, size_t ws_bytes, int32_t* status, void* stream);
+
+/* bsa_forward_noalloc — bsa_forward for callers that cannot allocate device memory.
+ * (No counterpart in the pages: this is a deployment variant of bsa_forward.)
+ * Some callers cannot call cudaMalloc: a host whose memory pool owns the whole device
+ * and forbids allocations from plug-ins, a serving loop that cannot take cudaMalloc's
+ * implicit synchronisation, an embedded runtime with a memory budget fixed at load time.
+ * This call takes the same arguments as bsa_forward minus the workspace and computes
+ * the same result; its scratch is one __device__ array of BSA_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library keeps until the process
+ * exits. It calls no allocating routine.
+ *   - The scratch address is looked up on the first call made on each device (with that
+ *     device current, and the stream on that device); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array (per device) and leaves its contents behind; calls
+ *     whose kernels overlap on the GPU (different streams or host threads) race on it,
+ *     so serialise them.
+ *   - Returns BSA_ERR_SCRATCH_LIMIT when the shape needs more scratch than the array
+ *     holds: PISA needs 256 + 2*BH*Mp*d*2 + BH*d*d*2 bytes (Mp = M rounded up to 128,
+ *     each term rounded up to 256), keep-or-drop 256 bytes. Other errors as bsa_forward. */
+BSA_API bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void* V, int32_t Bt,
+                                       int32_t H, int32_t L, int32_t d, int32_t block,
+                                       const int32_t* row_ptr, const int32_t* col_idx,
+                                       int64_t nnz_total, int32_t csr_per_head, int32_t mode,
+                                       const float* kbar, const float* vsum, const float* Hbar,
+                                       float scale, void* O, float* lse, int32_t* status,
+                                       void* stream);
 
 #ifdef __cplusplus
 }

@@ -21,13 +21,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsattn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_BAD_CSR, ERR_TIMEOUT, ERR_WORKSPACE, \
-    ERR_CAPACITY = range(8)
+    ERR_CAPACITY, ERR_SCRATCH_LIMIT = range(9)
+NOALLOC_SCRATCH_BYTES = 16 << 20
 MODE_KEEP_OR_DROP, MODE_PISA = 0, 1
 CALL_BUILD_MASK, CALL_PRECOMPUTE, CALL_ROUTE, CALL_FORWARD = 0, 1, 2, 3
 
 # Every symbol include/bsattn.h declares, in header order.
 EXPORTS = ("bsa_version", "bsa_status_string", "bsa_mask_blocks", "bsa_workspace_bytes",
-           "bsa_build_mask", "bsa_precompute", "bsa_route", "bsa_forward")
+           "bsa_build_mask", "bsa_precompute", "bsa_route", "bsa_forward",
+           "bsa_forward_noalloc")
 
 
 class BsaError(RuntimeError):
@@ -57,6 +59,8 @@ _SIGS = {
                          _vp, _vp, _vp, _vp]),
     "bsa_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _i32,
                            _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
+                                   _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -200,6 +204,30 @@ def bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum
                              _ptr(kbar), _ptr(vsum), _ptr(Hbar), float(scale), _ptr(O),
                              _ptr(lse), _ptr(workspace), ws_bytes, _ptr(status),
                              _stream(stream)), "bsa_forward")
+
+
+def bsa_forward_noalloc(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum, Hbar,
+                        scale, O, lse=None, status=None, stream=None):
+    """bsa_forward without a workspace argument: the library's built-in device scratch
+    array is used instead, for callers that cannot allocate device memory."""
+    Bt, H, L, d = _bhld(Q, "Q")
+    _need(K, torch.bfloat16, "K", Q.shape)
+    _need(V, torch.bfloat16, "V", Q.shape)
+    _need(O, torch.bfloat16, "O", Q.shape)
+    _need(row_ptr, torch.int32, "row_ptr")
+    _need(col_idx, torch.int32, "col_idx")
+    M = L // block
+    if mode == MODE_PISA:
+        _need(kbar, torch.float32, "kbar", (Bt * H, M, d))
+        _need(vsum, torch.float32, "vsum", (Bt * H, M, d))
+        _need(Hbar, torch.float32, "Hbar", (Bt * H, d, d))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", (Bt * H, L))
+    _check(lib().bsa_forward_noalloc(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block,
+                                     _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                     int(csr_per_head), int(mode), _ptr(kbar), _ptr(vsum),
+                                     _ptr(Hbar), float(scale), _ptr(O), _ptr(lse),
+                                     _ptr(status), _stream(stream)), "bsa_forward_noalloc")
 
 
 # ------------------------------------------------------------ allocating helpers

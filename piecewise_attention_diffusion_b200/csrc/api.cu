@@ -55,6 +55,7 @@ const char* bsa_status_string(int32_t code) {
     case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
     case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
     case BSA_ERR_CAPACITY: return "BSA_ERR_CAPACITY";
+    case BSA_ERR_SCRATCH_LIMIT: return "BSA_ERR_SCRATCH_LIMIT";
     default: return "BSA_UNKNOWN_STATUS";
   }
 }
