@@ -171,15 +171,23 @@ def peaks() -> dict:
 
 
 def load_traffic(w) -> float | None:
-    """DRAM bytes per launch of the forward kernel from the committed ncu summary of
-    the current kernel (None when no capture matches the current kernel)."""
+    """DRAM bytes per launch of the forward kernel from the committed ncu summary, only
+    while the kernel source is the one that was captured and the head count matches
+    (None otherwise: counters of another kernel do not describe this one)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    src = os.path.join(ROOT, "piecewise_attention_diffusion_b200", "csrc", "forward_tc.cu")
+    if not os.path.exists(p) or not os.path.exists(src):
         return None
     with open(p) as f:
-        d = json.load(f)
-    e = d.get(w.name)
-    return None if e is None else e.get("bytes_per_launch")
+        e = json.load(f).get(w.name)
+    if e is None or e.get("scaled_to_heads") != w.heads:
+        return None
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if not h.startswith(e.get("source_sha256_prefix", "?")):
+        return None
+    return e.get("bytes_per_launch")
 
 
 # -------------------------------------------------------------- CPU oracle timing
