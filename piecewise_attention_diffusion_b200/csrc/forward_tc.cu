@@ -193,9 +193,9 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const CUtensorMap* map = kind == 0 ? &tmK : kind == 1 ? &tmV : kind == 2 ? &tmKb
                                  : kind == 3 ? &tmVs : &tmHb;
         const int y = kind <= 1 ? j * BKV : (kind == 4 ? 0 : j * kChunk);
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(dst + h * rows * 128, map, &bars.kv_full[slot], h * 64, y, bh);
+        // one 4-D box: 64 columns x rows x (D/64) column groups; lands as D/64 swizzled
+        // [rows x 64] sub-tiles, sub-tile h at byte offset h * rows * 128
+        tma_load_4d(dst, map, &bars.kv_full[slot], 0, y, 0, bh);
         ++ring;
         (void)t_idx;
         return true;
@@ -208,9 +208,13 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const int qb = it & 1;
         if (!mbar_wait(&bars.q_empty[qb], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars.q_full[qb], p.qbox * D * 2);
+        if (p.qbox == kBQ) {
+          tma_load_4d(smem + qb * C::QBYTES, &tmQ, &bars.q_full[qb], 0, qt * kBQ, 0, bh);
+        } else {  // L < 128: one box per column group, at the 128-row sub-tile stride
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(smem + qb * C::QBYTES + h * kBQ * 128, &tmQ, &bars.q_full[qb], h * 64, qt * kBQ, bh);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + qb * C::QBYTES + h * kBQ * 128, &tmQ, &bars.q_full[qb], 0, 0, h, bh);
+        }
         ++q_issued;
         Lists lk = lists, lv = lists;
         for (int t = 0; t < n && ok; ++t) {
@@ -595,15 +599,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor [z][rows][cols] (cols contiguous), boxes of 64 columns x box_rows rows.
-bool make_map(CUtensorMap* m, const void* ptr, int cols, int rows, int z, int box_rows) {
+// bf16 tensor [z][rows][cols] (cols contiguous, cols a multiple of 64) viewed as 4-D
+// (64 columns, rows, cols/64 column groups, z) so that one box of 64 x box_rows x
+// cols/64 lands in shared memory as cols/64 consecutive [box_rows x 64] sub-tiles, each
+// 128-byte swizzled: the operand layout of the MMA descriptors (sub-tile h at byte
+// offset h * box_rows * 128). With all_groups false the box holds one column group, for
+// callers that place the groups themselves (a Q tile shorter than 128 rows).
+bool make_map(CUtensorMap* m, const void* ptr, int cols, int rows, int z, int box_rows,
+              bool all_groups = true) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)z};
-  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * rows * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)z};
+  cuuint64_t strides[3] = {(cuuint64_t)cols * 2, 128, (cuuint64_t)cols * rows * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, all_groups ? (cuuint32_t)(cols / 64) : 1u, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -625,7 +635,8 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmHb;
   const int qbox = s.L < kBQ ? s.L : kBQ;
   const int Mp = ceil_div(M, kChunk) * kChunk;
-  bool ok = make_map(&tmQ, a.Q, D, s.L, BH, qbox) && make_map(&tmK, a.K, D, s.L, BH, BKV) &&
+  bool ok = make_map(&tmQ, a.Q, D, s.L, BH, qbox, qbox == kBQ) &&
+            make_map(&tmK, a.K, D, s.L, BH, BKV) &&
             make_map(&tmV, a.V, D, s.L, BH, BKV);
   if (a.mode == BSA_MODE_PISA) {
     ok = ok && make_map(&tmKb, kb16, D, Mp, BH, kChunk) && make_map(&tmVs, vs16, D, Mp, BH, kChunk) &&

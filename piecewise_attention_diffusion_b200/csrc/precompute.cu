@@ -9,7 +9,8 @@
 //     H_j = sum_n (k_n - kbar_j)^T v_n = K_j^T V_j - kbar_j^T vsum_j,
 // so the d x d product K_j^T V_j runs on the tensor cores (bf16 in, fp32 accumulate)
 // and the centring is one fp32 rank-1 update. The kernels are HBM-bound (each block's
-// K and V are read once per pass); three launches:
+// K and V are read once per pass); three launches (this file serves d = 64; d = 128
+// runs on the tensor-core kernels of precompute_tc.cu):
 //   k_pre_stats : kbar, vsum, and partial sums of H_j over groups of G blocks;
 //   k_pre_reduce: Hbar = (1/M) * sum of the partials, in a fixed order (deterministic);
 //   k_pre_norm  : recompute H_j per block, Mnorm_j = ||H_j - Hbar||_F, optional H_j out.
@@ -278,6 +279,7 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
 }  // namespace
 
 size_t precompute_workspace(const Shape& s) {
+  if (s.d == 128) return precompute_tc_workspace(s);
   const int n_grp = ceil_div(s.M(), group_size(s));
   return (size_t)s.BH() * n_grp * s.d * s.d * sizeof(float);
 }
@@ -285,11 +287,12 @@ size_t precompute_workspace(const Shape& s) {
 cudaError_t launch_precompute(const Shape& s, const void* K, const void* V, float* kbar,
                               float* vsum, float* Hbar, float* Mnorm, float* Hblk, void* ws,
                               int32_t* status, cudaStream_t st) {
-  (void)status;
-  if (s.block == 64 && s.d == 64) return run<64, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
-  if (s.block == 64 && s.d == 128) return run<64, 128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
-  if (s.block == 128 && s.d == 64) return run<128, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
-  return run<128, 128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
+  // d = 128: tensor-core kernels (precompute_tc.cu); d = 64 (an M = 64 tcgen05 tile has a
+  // different TMEM layout) keeps the mma.sync kernels of this file
+  if (s.d == 128)
+    return launch_precompute_tc(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+  if (s.block == 64) return run<64, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
+  return run<128, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
 }
 
 }  // namespace bsa

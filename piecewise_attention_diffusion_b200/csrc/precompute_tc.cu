@@ -1,0 +1,447 @@
+// bsa_precompute for d = 128 on the tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers",
+// technical summary §2: per KV block j the centroid kbar_j, the value sum vsum_j and
+// the first-order matrix H_j = sum_n (k_{j,n} - kbar_j)^T v_{j,n}; H-bar is the mean of
+// the H_j over the head and routing uses M_j = ||H_j - H-bar||.
+//
+// Per block the tensor core computes, from the K_j and V_j tiles exactly as TMA lands
+// them (both operands MN-major, 128-byte swizzled):
+//     C_j    = K_j^T V_j                  (d x d, fp32 in TMEM)
+//     ksum_j = K_j^T 1,  vsum_j = V_j^T 1  (against a tile of ones: exact column sums)
+// and the epilogue thread that owns row a of C applies the centring in fp32:
+//     H_j[a][c] = C_j[a][c] - (ksum_j[a] / B) * vsum_j[c].
+// Two passes over K and V, because M_j needs H-bar, i.e. every block of the head:
+//   stats pass  writes kbar, vsum and, per group of kGroup blocks, the partial sum of
+//               H_j (the group's rows kept in registers; written once per group);
+//   (a reduce kernel then forms H-bar from the partials in a fixed order);
+//   norm pass   recomputes H_j and reduces ||H_j - H-bar||_F over the 128 rows.
+// Each pass is one persistent kernel over contiguous ranges of blocks (so a CTA meets
+// few heads and reloads H-bar rarely): warp 0 issues TMA into a 3-stage ring of (K_j,
+// V_j) pairs, warp 1 issues the MMAs into two TMEM buffers, warps 2-5 run the epilogue.
+// Every mbarrier wait is bounded; a timeout aborts the CTA and reports BSA_ERR_TIMEOUT.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace bsa {
+namespace pretc {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr int kGroup = 8;  // blocks per partial sum of H_j (stats pass)
+constexpr uint32_t kTmemCols = 512;
+// TMEM buffer b: C at 256 b, ksum at 256 b + 128, vsum at 256 b + 144 (16 columns each)
+
+template <int B>
+struct Cfg {
+  static constexpr int TILE = B * D * 2;       // one K or V tile
+  static constexpr int STAGE = 2 * TILE;       // K and V
+  static constexpr int ONES = 16 * B * 2;      // 16 x B tile of ones (K-major)
+  static constexpr int SMEM = kStages * STAGE + ONES + 1024;
+};
+
+struct Params {
+  int L, M, BH;
+  int n_units, per_cta;   // units: groups of kGroup blocks (stats) or blocks (norm)
+  bool stats;             // unit = group of kGroup blocks (stats pass) or one block
+  float* kbar;
+  float* vsum;
+  float* partial;         // stats: [BH, ceil(M / kGroup), D, D]
+  const float* Hbar;      // norm
+  float* Mnorm;           // norm
+  float* Hblk;            // norm, nullable
+  int32_t* status;
+};
+
+// The blocks this CTA processes, in order: unit range [u0, u1) of the pass.
+struct BlockIter {
+  int u, u1, j, j1, bh;
+  bool stats;
+  int M, n_grp;
+  __device__ __forceinline__ void init(const Params& p) {
+    stats = p.stats;
+    M = p.M;
+    n_grp = ceil_div(p.M, kGroup);
+    u = blockIdx.x * p.per_cta;
+    u1 = min(p.n_units, u + p.per_cta);
+    j = j1 = 0;
+    bh = 0;
+    load_unit();
+  }
+  __device__ __forceinline__ void load_unit() {
+    if (u >= u1) return;
+    if (stats) {
+      bh = u / n_grp;
+      const int g = u % n_grp;
+      j = g * kGroup;
+      j1 = min(M, j + kGroup);
+    } else {
+      bh = u / M;
+      j = u % M;
+      j1 = j + 1;
+    }
+  }
+  __device__ __forceinline__ bool valid() const { return u < u1; }
+  // advance to the next block; returns true when a unit (group) just ended
+  __device__ __forceinline__ bool next() {
+    ++j;
+    if (j < j1) return false;
+    ++u;
+    load_unit();
+    return true;
+  }
+};
+
+struct Barriers {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t mma_done[2], tmem_free[2], xch[2], xred[2];
+  uint64_t done;
+};
+
+template <int B, bool kStats>
+__global__ void __launch_bounds__(kThreads, 1)
+k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+             const Params p) {
+  using C = Cfg<B>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sOnes = smem + kStages * C::STAGE;
+  __shared__ Barriers bars;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float s_vs[2][D];
+  __shared__ float s_red[2][4];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // ones tile (its swizzle is irrelevant: every element is 1.0)
+  for (int e = threadIdx.x; e < C::ONES / 4; e += kThreads)
+    reinterpret_cast<uint32_t*>(sOnes)[e] = 0x3F803F80u;  // bf16 pair (1.0, 1.0)
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&bars.full[i], 1);
+      mbar_init(&bars.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.mma_done[i], 1);
+      mbar_init(&bars.tmem_free[i], 128);
+      mbar_init(&bars.xch[i], 128);
+      mbar_init(&bars.xred[i], 128);
+    }
+    mbar_init(&bars.done, 1);
+    fence_barrier_init();
+  }
+  // the ones tile is read by the tensor core (async proxy)
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+
+  if (warp == 0) {
+    // ============================================================== TMA producer
+    if (lane == 0) {
+      BlockIter it;
+      it.init(p);
+      uint32_t n = 0;
+      bool ok = true;
+      while (it.valid()) {
+        const int st = n % kStages;
+        if (!(ok = mbar_wait(&bars.empty[st], ((n / kStages) & 1) ^ 1, abort_flag))) break;
+        unsigned char* dst = smem + st * C::STAGE;
+        mbar_arrive_expect_tx(&bars.full[st], C::STAGE);
+        tma_load_4d(dst, &tmK, &bars.full[st], 0, it.j * B, 0, it.bh);
+        tma_load_4d(dst + C::TILE, &tmV, &bars.full[st], 0, it.j * B, 0, it.bh);
+        ++n;
+        it.next();
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        const uint32_t first = n > (uint32_t)kStages ? n - kStages : 0;
+        for (uint32_t r = first; r < n; ++r)
+          while (!mbar_try_wait(&bars.full[r % kStages], (r / kStages) & 1) &&
+                 globaltimer_ns() - t0 < 100000000ull) {
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_c = idesc_bf16_f32(128, D, true, true);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, true, false);
+      const uint32_t ones = smem_u32(sOnes);
+      BlockIter it;
+      it.init(p);
+      uint32_t n = 0;
+      bool ok = true;
+      while (it.valid()) {
+        const int st = n % kStages, b = n & 1;
+        ok = mbar_wait(&bars.full[st], (n / kStages) & 1, abort_flag);
+        if (ok && n >= 2) ok = mbar_wait(&bars.tmem_free[b], ((n >> 1) - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + st * C::STAGE);
+        const uint32_t v_addr = k_addr + C::TILE;
+        const uint32_t dc = tmem + 256u * b;
+#pragma unroll
+        for (int k = 0; k < B / 16; ++k) {
+          const uint64_t a_k = smem_desc_sw128(k_addr + k * 2048, B * 128, 1024);
+          const uint64_t a_v = smem_desc_sw128(v_addr + k * 2048, B * 128, 1024);
+          const uint64_t b_o = smem_desc_sw128(ones + (k / 4) * (16 * 128) + (k % 4) * 32, 16, 1024);
+          mma_ss(dc, a_k, a_v, idesc_c, k > 0 ? 1u : 0u);          // K^T V
+          mma_ss(dc + 128, a_k, b_o, idesc_s, k > 0 ? 1u : 0u);    // K^T 1
+          mma_ss(dc + 144, a_v, b_o, idesc_s, k > 0 ? 1u : 0u);    // V^T 1
+        }
+        mma_commit(&bars.empty[st]);
+        mma_commit(&bars.mma_done[b]);
+        ++n;
+        it.next();
+      }
+      mma_commit(&bars.done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&bars.done, 0) && globaltimer_ns() - t0 < 100000000ull) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================== epilogue
+    const int quad = warp % 4;
+    const int a = quad * 32 + lane;              // row of C = TMEM lane
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const int n_grp = ceil_div(p.M, kGroup);
+    // stats: partial sum of H_j row a over the group; norm: H-bar row a of the head
+    float acc[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    int hb_head = -1;
+    BlockIter it;
+    it.init(p);
+    uint32_t n = 0;
+    bool ok = true;
+    while (it.valid()) {
+      const int b = n & 1;
+      const uint32_t ph = (n >> 1) & 1;
+      const int bh = it.bh, j = it.j;
+      if (!kStats && bh != hb_head) {
+        const float4* src = reinterpret_cast<const float4*>(p.Hbar + ((size_t)bh * D + a) * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) {
+          const float4 v = __ldg(src + c);
+          acc[4 * c] = v.x;
+          acc[4 * c + 1] = v.y;
+          acc[4 * c + 2] = v.z;
+          acc[4 * c + 3] = v.w;
+        }
+        hb_head = bh;
+      }
+      ok = mbar_wait(&bars.mma_done[b], ph, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t base = tmem + lane_addr + 256u * b;
+      float kb, vs;
+      {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(base + 128, r0);
+        tmem_ld16(base + 144, r1);
+        tmem_wait_ld();
+        kb = __uint_as_float(r0[0]) * (1.0f / B);
+        vs = __uint_as_float(r1[0]);
+      }
+      if (kStats) {
+        const size_t o = ((size_t)bh * p.M + j) * D + a;
+        p.kbar[o] = kb;
+        p.vsum[o] = vs;
+      }
+      // every row needs vsum_j[c] for all c: exchange through shared memory
+      s_vs[b][a] = vs;
+      mbar_arrive(&bars.xch[b]);
+      ok = mbar_wait(&bars.xch[b], ph, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      float sq = 0.f;
+      float* hrow = (!kStats && p.Hblk) ? p.Hblk + (((size_t)bh * p.M + j) * D + a) * D : nullptr;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(base + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float h = fmaf(-kb, s_vs[b][c0 + e], __uint_as_float(r[e]));
+          if (kStats) {
+            acc[c0 + e] += h;
+          } else {
+            const float dlt = h - acc[c0 + e];
+            sq = fmaf(dlt, dlt, sq);
+            r[e] = __float_as_uint(h);
+          }
+        }
+        if (hrow) {
+          float4* dst = reinterpret_cast<float4*>(hrow + c0);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+      }
+      // the TMEM buffer is free for the block after next
+      tc_fence_before();
+      mbar_arrive(&bars.tmem_free[b]);
+      if (!kStats) {
+        sq = warp_sum(sq);
+        if (lane == 0) s_red[b][quad] = sq;
+        mbar_arrive(&bars.xred[b]);
+        ok = mbar_wait(&bars.xred[b], ph, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (a == 0)
+          p.Mnorm[(size_t)bh * p.M + j] =
+              sqrtf((s_red[b][0] + s_red[b][1]) + (s_red[b][2] + s_red[b][3]));
+      }
+      ++n;
+      const bool unit_end = it.next();
+      if (kStats && unit_end) {
+        // group finished: write its partial sum (row a) and start a new one
+        const int g = j / kGroup;
+        float4* dst = reinterpret_cast<float4*>(p.partial + (((size_t)bh * n_grp + g) * D + a) * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) {
+          dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+          acc[4 * c] = acc[4 * c + 1] = acc[4 * c + 2] = acc[4 * c + 3] = 0.f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_sh) report(p.status, BSA_ERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// H-bar = (1 / M) * sum of the partial sums of one head, in a fixed order.
+__global__ void k_reduce(const float* __restrict__ partial, int n_grp, int M,
+                         float* __restrict__ Hbar) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int bh = blockIdx.y;
+  if (e >= D * D) return;
+  const float* q = partial + (size_t)bh * n_grp * D * D + e;
+  float s = 0.f;
+  for (int g = 0; g < n_grp; ++g) s += q[(size_t)g * D * D];
+  Hbar[(size_t)bh * D * D + e] = s / (float)M;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// K or V [BH][L][D] as 4-D (64 columns, L rows, D/64 groups, BH): one box = one block tile
+// landing as D/64 swizzled [B x 64] sub-tiles.
+bool make_map(CUtensorMap* m, const void* ptr, int L, int BH, int B) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)L, (cuuint64_t)(D / 64), (cuuint64_t)BH};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)D * L * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)B, (cuuint32_t)(D / 64), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int B>
+cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float* vsum,
+                float* Hbar, float* Mnorm, float* Hblk, void* ws, int32_t* status,
+                cudaStream_t st) {
+  using Cf = Cfg<B>;
+  CUtensorMap tmK, tmV;
+  if (!make_map(&tmK, K, s.L, s.BH(), B) || !make_map(&tmV, V, s.L, s.BH(), B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_precompute<B, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_precompute<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  const int M = s.M(), n_grp = ceil_div(M, kGroup), sms = sm_count();
+  Params p;
+  p.L = s.L;
+  p.M = M;
+  p.BH = s.BH();
+  p.kbar = kbar;
+  p.vsum = vsum;
+  p.partial = static_cast<float*>(ws);
+  p.Hbar = Hbar;
+  p.Mnorm = Mnorm;
+  p.Hblk = Hblk;
+  p.status = status;
+  // stats pass over groups of kGroup blocks
+  p.stats = true;
+  p.n_units = s.BH() * n_grp;
+  p.per_cta = ceil_div(p.n_units, sms);
+  k_precompute<B, true><<<ceil_div(p.n_units, p.per_cta), kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_reduce<<<dim3(ceil_div(D * D, 256), s.BH()), 256, 0, st>>>(p.partial, n_grp, M, Hbar);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // norm pass over single blocks
+  p.stats = false;
+  p.n_units = s.BH() * M;
+  p.per_cta = ceil_div(p.n_units, sms);
+  k_precompute<B, false><<<ceil_div(p.n_units, p.per_cta), kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace pretc
+
+size_t precompute_tc_workspace(const Shape& s) {
+  return (size_t)s.BH() * ceil_div(s.M(), pretc::kGroup) * pretc::D * pretc::D * sizeof(float);
+}
+
+cudaError_t launch_precompute_tc(const Shape& s, const void* K, const void* V, float* kbar,
+                                 float* vsum, float* Hbar, float* Mnorm, float* Hblk, void* ws,
+                                 int32_t* status, cudaStream_t st) {
+  if (s.block == 64)
+    return pretc::run<64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+  return pretc::run<128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+}
+
+}  // namespace bsa

@@ -8,29 +8,26 @@
 //     score_ij = softmax_j(s * qbar_i . kbar_j) + lambda * M_j / sum_j' M_j'
 // (two distributions, so the mix is scale-free), qbar_i the mean query of block i.
 //
-// One CTA per (head, query block). The query block is read once with 16-byte loads
-// (the only HBM stream; kbar and Mnorm are small and L2-resident), the M block scores
-// are warp dot products, and the top-k is an exact rank count with ties broken towards
-// the smaller index, compacted in ascending order with a ballot scan.
+// One CTA per (head, 8 query blocks), one warp per query block:
+//   1. pooled query: the warp streams its block of Q with 16-byte loads (the only HBM
+//      stream of the call) and reduces the columns;
+//   2. scores: the head's centroids are staged through shared memory in chunks of 64
+//      rows (rows padded to D+1 floats so that 32 lanes reading 32 centroids hit 32
+//      banks) and each lane dots its centroids with the pooled query;
+//   3. softmax over the M blocks plus the normalised covariance term;
+//   4. exact top-k: the k-th largest score is found by a radix select on the float bit
+//      patterns (scores are >= 0, so the bit patterns order like the values), ties at
+//      the threshold go to the smaller block index, and the selected indices are
+//      compacted in ascending order with ordered ballots.
 #include "common.cuh"
 #include "internal.h"
 
 namespace bsa {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
-
-__device__ __forceinline__ float block_reduce(float v, float* s_tmp, bool is_max) {
-  v = is_max ? warp_max(v) : warp_sum(v);
-  const int w = threadIdx.x / 32;
-  __syncthreads();
-  if (threadIdx.x % 32 == 0) s_tmp[w] = v;
-  __syncthreads();
-  float r = s_tmp[0];
-  for (int i = 1; i < kWarps; ++i) r = is_max ? fmaxf(r, s_tmp[i]) : r + s_tmp[i];
-  return r;
-}
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunkC = 64;  // centroids per staged chunk
 
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
@@ -39,101 +36,137 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
         int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
         float* __restrict__ scores) {
   const int M = L / B;
-  const int i = blockIdx.x, bh = blockIdx.y;
-  extern __shared__ float s_buf[];
-  float* s_qbar = s_buf;                 // D
-  float* s_score = s_qbar + D;           // M
-  float* s_tmp = s_score + M;            // 32
-  float* s_part = s_tmp + 32;            // (kThreads / (D/8)) x D partial column sums
-  int* s_wcount = reinterpret_cast<int*>(s_part + kThreads / (D / 8) * D);  // kWarps
-
-  // 1. pooled query: column means over the B rows of block i
-  constexpr int CPR = D / 8;               // 16-byte chunks per row
-  constexpr int RG = kThreads / CPR;       // row groups
-  const int cc = threadIdx.x % CPR, rg = threadIdx.x / CPR;
-  const __nv_bfloat16* qb = Q + ((size_t)bh * L + (size_t)i * B) * D;
-  float part[8] = {};
-  for (int r = rg; r < B; r += RG) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(qb + (size_t)r * D) + cc);
-    float f[8];
-    bf16x8_to_f32(u, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) part[e] += f[e];
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) s_part[rg * D + cc * 8 + e] = part[e];
-  __syncthreads();
-  for (int c = threadIdx.x; c < D; c += kThreads) {
-    float s = 0.f;
-    for (int g = 0; g < RG; ++g) s += s_part[g * D + c];
-    s_qbar[c] = s * (1.0f / B);
-  }
-  __syncthreads();
-
-  // 2. block scores a_j = scale * qbar . kbar_j
+  const int bh = blockIdx.y;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const float* kb = kbar + (size_t)bh * M * D;
-  for (int j = warp; j < M; j += kWarps) {
-    float s = 0.f;
-#pragma unroll
-    for (int c = lane; c < D; c += 32) s += s_qbar[c] * __ldg(kb + (size_t)j * D + c);
-    s = warp_sum(s);
-    if (lane == 0) s_score[j] = scale * s;
-  }
-  __syncthreads();
+  const int i = blockIdx.x * kWarps + warp;  // this warp's query block
+  const bool active = i < M;
 
-  // 3. softmax over the M blocks, plus the normalised covariance term
-  float mx = -INFINITY;
-  for (int j = threadIdx.x; j < M; j += kThreads) mx = fmaxf(mx, s_score[j]);
-  mx = block_reduce(mx, s_tmp, true);
-  float se = 0.f, sm = 0.f;
+  extern __shared__ float smem[];
+  float* s_kb = smem;                           // kChunkC x (D + 1)
+  float* s_q = s_kb + kChunkC * (D + 1);        // kWarps x D
+  float* s_cov = s_q + kWarps * D;              // M
+  float* s_sc = s_cov + M;                      // kWarps x M
+  float* s_red = s_sc + kWarps * M;             // kWarps
+
+  // normalised covariance term, shared by every query block of the head
   const float* mn = Mnorm + (size_t)bh * M;
-  for (int j = threadIdx.x; j < M; j += kThreads) {
-    se += expf(s_score[j] - mx);
-    sm += __ldg(mn + j);
-  }
-  se = block_reduce(se, s_tmp, false);
-  sm = block_reduce(sm, s_tmp, false);
-  const float inv_se = 1.0f / se;
-  const float cov = sm > 0.f ? lambda / sm : 0.f;
+  float part = 0.f;
+  for (int j = threadIdx.x; j < M; j += kThreads) part += __ldg(mn + j);
+  part = warp_sum(part);
+  if (lane == 0) s_red[warp] = part;
   __syncthreads();
-  for (int j = threadIdx.x; j < M; j += kThreads) {
-    const float sc = expf(s_score[j] - mx) * inv_se + cov * __ldg(mn + j);
-    s_score[j] = sc;
-    if (scores) scores[((size_t)bh * M + i) * M + j] = sc;
-  }
-  __syncthreads();
+  float msum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) msum += s_red[w];
+  const float cov = msum > 0.f ? lambda / msum : 0.f;
+  for (int j = threadIdx.x; j < M; j += kThreads) s_cov[j] = cov * __ldg(mn + j);
 
-  // 4. exact top-k by rank count; 5. ascending compaction with a ballot scan
-  const int64_t head_base = (int64_t)bh * M * k_top;
-  int base = 0;
-  for (int j0 = 0; j0 < M; j0 += kThreads) {
-    const int j = j0 + threadIdx.x;
-    bool sel = false;
-    if (j < M) {
-      const float sj = s_score[j];
-      int rank = 0;
-      for (int jj = 0; jj < M; ++jj) {
-        const float o = s_score[jj];
-        rank += (o > sj || (o == sj && jj < j)) ? 1 : 0;
-      }
-      sel = rank < k_top;
+  // 1. pooled query of block i: lanes 0..CPR-1 take row r, the next CPR lanes row r+1...
+  constexpr int CPR = D / 8;          // 16-byte chunks per row
+  constexpr int RPI = 32 / CPR;       // rows per warp iteration
+  float* qbar = s_q + warp * D;
+  if (active) {
+    const __nv_bfloat16* qb = Q + ((size_t)bh * L + (size_t)i * B) * D;
+    const int cc = lane % CPR, r0 = lane / CPR;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int r = r0; r < B; r += RPI) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(qb + (size_t)r * D) + cc);
+      float f[8];
+      bf16x8_to_f32(u, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[e];
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) s_wcount[warp] = __popc(bal);
-    __syncthreads();
-    int pos = base + __popc(bal & ((1u << lane) - 1u));
-    for (int w = 0; w < warp; ++w) pos += s_wcount[w];
-    if (sel) col_idx[head_base + (int64_t)i * k_top + pos] = j;
-    int tot = 0;
-    for (int w = 0; w < kWarps; ++w) tot += s_wcount[w];
-    base += tot;
-    __syncthreads();
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane < CPR) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qbar[cc * 8 + e] = acc[e] * (1.0f / B);
+    }
   }
-  if (threadIdx.x == 0) {
+  __syncwarp();
+
+  // 2. block scores a_j = scale * qbar . kbar_j, centroids staged 64 at a time
+  const float* kb = kbar + (size_t)bh * M * D;
+  float* sc = s_sc + warp * M;
+  for (int c0 = 0; c0 < M; c0 += kChunkC) {
+    const int nc = min(kChunkC, M - c0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < nc * D; e += kThreads) {
+      const int r = e / D, c = e % D;
+      s_kb[r * (D + 1) + c] = __ldg(kb + (size_t)(c0 + r) * D + c);
+    }
+    __syncthreads();
+    if (active) {
+      for (int jj = lane; jj < nc; jj += 32) {
+        const float* kr = s_kb + jj * (D + 1);
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < D; c += 4) {
+          d0 = fmaf(qbar[c], kr[c], d0);
+          d1 = fmaf(qbar[c + 1], kr[c + 1], d1);
+          d2 = fmaf(qbar[c + 2], kr[c + 2], d2);
+          d3 = fmaf(qbar[c + 3], kr[c + 3], d3);
+        }
+        sc[c0 + jj] = scale * ((d0 + d1) + (d2 + d3));
+      }
+    }
+  }
+  __syncwarp();
+  if (!active) return;
+
+  // 3. softmax over the M blocks plus the covariance term
+  float mx = -INFINITY;
+  for (int j = lane; j < M; j += 32) mx = fmaxf(mx, sc[j]);
+  mx = warp_max(mx);
+  float se = 0.f;
+  for (int j = lane; j < M; j += 32) se += expf(sc[j] - mx);
+  se = warp_sum(se);
+  const float inv_se = 1.0f / se;
+  float* srow = scores ? scores + ((size_t)bh * M + i) * M : nullptr;
+  for (int j = lane; j < M; j += 32) {
+    const float v = expf(sc[j] - mx) * inv_se + s_cov[j];
+    sc[j] = v;
+    if (srow) srow[j] = v;
+  }
+  __syncwarp();
+
+  // 4. k-th largest key (bit pattern of a non-negative float) by radix select
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int cnt = 0;
+    for (int j = lane; j < M; j += 32) cnt += __float_as_uint(sc[j]) >= cand ? 1 : 0;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= k_top) T = cand;
+  }
+  int greater = 0;
+  for (int j = lane; j < M; j += 32) greater += __float_as_uint(sc[j]) > T ? 1 : 0;
+  greater = __reduce_add_sync(0xffffffffu, greater);
+  const int ties_needed = k_top - greater;  // >= 1
+
+  // 5. ascending compaction: selected = key > T, or key == T among the first
+  //    ties_needed such keys in index order
+  const int64_t base = (int64_t)bh * M * k_top + (int64_t)i * k_top;
+  const unsigned lt = (1u << lane) - 1u;
+  int ties_seen = 0, out = 0;
+  for (int j0 = 0; j0 < M; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < M ? __float_as_uint(sc[j]) : 0u;
+    const bool tie = j < M && key == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const bool sel = j < M && (key > T || (tie && ties_seen + __popc(tb & lt) < ties_needed));
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) col_idx[base + out + __popc(sb & lt)] = j;
+    ties_seen += __popc(tb);
+    out += __popc(sb);
+  }
+  if (lane == 0) {
     int32_t* rp = row_ptr + (size_t)bh * (M + 1);
-    rp[i] = (int32_t)(head_base + (int64_t)i * k_top);
-    if (i == M - 1) rp[M] = (int32_t)(head_base + (int64_t)M * k_top);
+    rp[i] = (int32_t)base;
+    if (i == M - 1) rp[M] = (int32_t)((int64_t)bh * M * k_top + (int64_t)M * k_top);
   }
 }
 
@@ -142,12 +175,13 @@ cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* M
                 int k_top, float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
                 float* scores, cudaStream_t st) {
   const int M = s.M();
-  const size_t sm = (D + M + 32 + (size_t)kThreads / (D / 8) * D) * sizeof(float) +
-                    kWarps * sizeof(int);
+  const size_t sm =
+      ((size_t)kChunkC * (D + 1) + (size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) *
+      sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(k_route<B, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  k_route<B, D><<<dim3(M, s.BH()), kThreads, sm, st>>>(
+  k_route<B, D><<<dim3(ceil_div(M, kWarps), s.BH()), kThreads, sm, st>>>(
       static_cast<const __nv_bfloat16*>(Q), kbar, Mnorm, s.L, k_top, lambda, scale, row_ptr,
       col_idx, scores);
   return cudaGetLastError();

@@ -204,7 +204,7 @@ def test_forward_multimodal_fixed_mask_keep_or_drop():
                    heads_idx=[0, 17, 63, 127])
 
 
-@pytest.mark.parametrize("L,block,d,kk", [(576, 64, 64, 3), (640, 128, 128, 2),
+@pytest.mark.parametrize("L,block,d,kk", [(576, 64, 64, 3), (640, 128, 128, 2), (64, 64, 128, 1),
                                           (128, 128, 128, 1), (64, 64, 64, 1),
                                           (1152, 64, 128, 5), (768, 128, 64, 6)])
 @pytest.mark.parametrize("mode", [b.MODE_KEEP_OR_DROP, b.MODE_PISA])
