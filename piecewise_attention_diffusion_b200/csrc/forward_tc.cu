@@ -11,19 +11,28 @@
 //   first order      (PISA) T = Q Hbar on the tensor cores; the epilogue writes
 //                    o = (O + s * sum_alpha * T) / l.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialised):
-//   warp 0  TMA producer: Q tiles (double-buffered) and a 4-slot ring of K / V /
-//           centroid / Hbar tiles, each 128-byte swizzled, completion on mbarriers;
-//   warp 1  MMA issuer (one thread): S = Q K^T into TMEM (two S buffers so the next
-//           QK^T runs while the softmax works on the current one), O += P V with P read
-//           from TMEM (bf16, aliased onto its own S buffer), T = Q Hbar;
-//   warps 2-5  softmax: thread r owns query row r (TMEM lane r); loads its S row with
-//           tcgen05.ld, applies the masks, exponentiates with ex2 in the log2 domain and
-//           writes P back with tcgen05.st. O is rescaled in TMEM only when the running
-//           max grows by more than 2^8 (the bound keeps every P <= 256, safe in bf16 and
-//           fp32), so most tiles need no correction pass. The same warps run the
-//           epilogue.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D), T [256+D, 256+2D).
+// Design (one persistent CTA per SM, 384 threads, warp-specialised, two query tiles in
+// flight so that the softmax of one overlaps the tensor-core work of the other):
+//   warps 0-3, 4-7  one softmax warpgroup per stream: thread r owns query row r (TMEM
+//           lane r). The whole S row is loaded into registers with one wait; the row max
+//           uses three-input max; P = 2^(s*scale*log2(e) - m) is formed with packed f32x2
+//           arithmetic, a quarter of the exponentials on the FMA pipe (polynomial) and the
+//           rest on the special-function unit, so that neither pipe limits alone; P goes
+//           back into TMEM as bf16 pairs with tcgen05.st. O is rescaled in TMEM only when
+//           the running max grows by more than 2^8 (keeps every P <= 256, safe in bf16 and
+//           fp32). The same warps run the epilogue and load the next query tile of their
+//           stream;
+//   warp 8  TMA producer of a ring of K / V / centroid / Hbar tiles (128-byte swizzled,
+//           completion on mbarriers), in the same step order as the MMA issuer;
+//   warp 9  MMA issuer (one thread), alternating one step of each stream:
+//           step 0 = S(0); step t = O += P(t-1) V(t-1), then S(t) = Q K(t)^T; last step =
+//           O += P(n-1) V(n-1) [, T = Q Hbar]. P is bf16 in TMEM over its own S buffer and
+//           is the A operand of the PV product. Because S(t) is issued after PV(t-1) in
+//           the same stream, S(t) being ready implies PV(t-1) has completed;
+//   warps 10-11  idle (they complete the control warpgroup, whose registers setmaxnreg
+//           hands to the softmax warpgroups).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D); the
+// first-order product T of a stream is written into its S buffer after its last PV.
 // Query tiles are 128 rows: one query block of 128, or two of 64 whose key-block lists
 // are merged (each row masks the key blocks its own block does not select).
 // Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA drains its
@@ -43,9 +52,23 @@ using namespace sm100;
 
 constexpr int kBQ = 128;       // query rows per tile
 constexpr int kChunk = 128;    // centroids per sweep tile
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kStreams = 2;                   // query tiles in flight per CTA
+constexpr int kThreads = 128 * (kStreams + 1);  // softmax warpgroups, then a control warpgroup
+constexpr int kProducerWarp = 4 * kStreams;      // first warp of the control warpgroup
+constexpr int kMmaWarp = kProducerWarp + 1;      // (its two other warps only idle)
+// Register split: the launch gives every thread 168 registers (3 warps per SMSP); the
+// control warpgroup drops to 88 and the softmax warpgroups rise to 208, which hold a whole
+// S row: 128 x 88 + 256 x 208 = 384 x 168.
+constexpr int kRegsControl = 88;
+constexpr int kRegsSoftmax = 208;
+static_assert(128 * kRegsControl + 128 * kStreams * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef BSA_POLY_OF8
+#define BSA_POLY_OF8 2
+#endif
+// pairs of exponentials, of every 8 pairs of an exact tile, computed on the FMA pipe
+constexpr int kPolyOf8 = BSA_POLY_OF8;
 
 struct Params {
   int L, M, BH, n_qt, n_items;
@@ -66,10 +89,11 @@ struct Cfg {
   static constexpr int QBPT = kBQ / BKV;          // query blocks per tile (1 or 2)
   static constexpr int QBYTES = kBQ * D * 2;
   static constexpr int SLOT = kBQ * D * 2;        // a slot holds up to 128 rows x D
-  static constexpr int NSLOT = D == 128 ? 4 : 8;
-  static constexpr int SMEM = 2 * QBYTES + NSLOT * SLOT + 1024;
-  static constexpr uint32_t O_COL = 256u;
-  static constexpr uint32_t T_COL = 256u + D;
+  static constexpr int NSLOT = D == 128 ? 5 : 8;
+  static constexpr int SMEM = kStreams * QBYTES + NSLOT * SLOT + 1024;
+  // TMEM columns: S of stream x at 128x, O of stream x at 256 + D*x
+  __host__ __device__ static constexpr uint32_t S_COL(int x) { return 128u * x; }
+  __host__ __device__ static constexpr uint32_t O_COL(int x) { return 256u + D * x; }
 };
 
 // The key-block lists of the (one or two) query blocks of a tile, merged ascending.
@@ -111,11 +135,98 @@ __device__ __forceinline__ int count_exact(Lists l) {
   return n;
 }
 
+// Work item k of stream x of this CTA (static schedule: the CTA takes items
+// blockIdx.x, blockIdx.x + G, ... and deals them to its two streams alternately).
+__device__ __forceinline__ int stream_item(int k, int x) {
+  return blockIdx.x + (2 * k + x) * gridDim.x;
+}
+
+// Per-stream position in the step schedule shared by the producer and the MMA issuer.
+// Steps of an item with n tiles: step 0 = S(0); step t (1 <= t < n) = PV(t-1), S(t);
+// step n = PV(n-1) [+ T] and the end of the item. An item with n = 0 has one step.
+template <int QBPT>
+struct StreamPos {
+  int k, item, bh, qt, n, n_ex, t;
+  uint32_t tiles;  // tiles of earlier items of this stream (barrier phases)
+  int items;       // earlier items of this stream
+  Lists lk, lv;    // K-side and V-side list cursors (producer)
+  __device__ __forceinline__ void start(const Params& p, int x, int n_ch) {
+    item = stream_item(k, x);
+    if (item >= p.n_items) return;
+    bh = item / p.n_qt;
+    qt = item % p.n_qt;
+    lk = item_lists<QBPT>(p, bh, qt);
+    lv = lk;
+    n_ex = count_exact<QBPT>(lk);
+    n = n_ex + n_ch;
+    t = 0;
+  }
+  __device__ __forceinline__ bool active(const Params& p) const { return item < p.n_items; }
+  __device__ __forceinline__ void advance(const Params& p, int x, int n_ch) {
+    tiles += n;
+    ++items;
+    ++k;
+    start(p, x, n_ch);
+  }
+};
+
+// Row max of the first N columns held in registers: three-input max in four chains.
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&r)[128]) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < N; e += 8) {
+    m0 = max3(m0, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+    m1 = max3(m1, __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+    m2 = max3(m2, __uint_as_float(r[e + 4]), __uint_as_float(r[e + 5]));
+    m3 = max3(m3, __uint_as_float(r[e + 6]), __uint_as_float(r[e + 7]));
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// P for one row: 2^(s * scale_log2 - m_ref) for the first N columns in r, written to TMEM
+// as bf16 pairs (column c holds elements 2c and 2c + 1) at p_addr; returns the fp32 row
+// sum. With kMixed, kPolyOf8 of every 8 pairs are computed on the FMA pipe (ex2_poly2)
+// and the rest on the special-function unit, so that the two pipes share the work; a row
+// that may hold -inf (masked centroids) uses the special-function unit only.
+template <int N, bool kMixed>
+__device__ __forceinline__ float row_exp(const uint32_t (&r)[128], float scale_log2,
+                                         float m_ref, uint32_t p_addr) {
+  const float2 sc = make_float2(scale_log2, scale_log2);
+  const float2 nm = make_float2(-m_ref, -m_ref);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int h = 0; h < N / 64; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int e = h * 64 + 2 * q;
+      const float2 xx =
+          fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sc, nm);
+      float2 ev;
+      if (kMixed && (q % 8) < kPolyOf8) {
+        ev = ex2_poly2(xx);
+      } else {
+        ev = make_float2(ex2(xx.x), ex2(xx.y));
+      }
+      acc[q & 3] = add2(acc[q & 3], ev);
+      pk[q] = pack_bf16x2(ev.x, ev.y);
+    }
+    tmem_st32(p_addr + h * 32, pk);
+  }
+  const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+  return a.x + a.y;
+}
+
+enum LoadKind { kLoadK = 0, kLoadV = 1, kLoadKbar = 2, kLoadVsum = 3, kLoadHbar = 4 };
+
 struct Barriers {
-  uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[8], kv_empty[8];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_bar, o_final, o_free, done;
+  uint64_t q_full[kStreams];
+  uint64_t s_full[kStreams], p_full[kStreams];
+  uint64_t o_final[kStreams], o_free[kStreams];
+  uint64_t done;
 };
 
 template <int D, int BKV>
@@ -130,7 +241,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sSlot = smem + 2 * C::QBYTES;
+  unsigned char* sSlot = smem + kStreams * C::QBYTES;
   __shared__ Barriers bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -138,27 +249,25 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     abort_sh = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.q_full[i], 1);
-      mbar_init(&bars.q_empty[i], 1);
-      mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.p_full[i], 128);
+    for (int x = 0; x < kStreams; ++x) {
+      mbar_init(&bars.q_full[x], 1);
+      mbar_init(&bars.s_full[x], 1);
+      mbar_init(&bars.p_full[x], 128);
+      mbar_init(&bars.o_final[x], 1);
+      mbar_init(&bars.o_free[x], 128);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(&bars.kv_full[i], 1);
       mbar_init(&bars.kv_empty[i], 1);
     }
-    mbar_init(&bars.o_bar, 1);
-    mbar_init(&bars.o_final, 1);
-    mbar_init(&bars.o_free, 128);
     mbar_init(&bars.done, 1);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&tmem_base_sh, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
@@ -174,64 +283,67 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
   const int n_ch = p.pisa ? ceil_div(p.M, kChunk) : 0;
-
-  if (warp == 0) {
-    // =============================================================== TMA producer
+  if (warp >= kProducerWarp) {
+  setmaxnreg_dec<kRegsControl>();
+  if (warp == kProducerWarp) {
+    // ================================================= TMA producer of the K/V ring
     if (lane == 0) {
       uint32_t ring = 0;
-      int it = 0;
-      int q_issued = 0;
       bool ok = true;
-      auto load_slot = [&](int kind, int t_idx, int j, int bh) -> bool {
-        // kind 0: K block j, 1: V block j, 2: centroid chunk, 3: value-sum chunk, 4: Hbar
+      auto tile_map = [&](int kind, int j, const CUtensorMap*& map, int& y, int& rows) {
+        map = kind == kLoadK ? &tmK : kind == kLoadV ? &tmV : kind == kLoadKbar ? &tmKb
+              : kind == kLoadVsum ? &tmVs : &tmHb;
+        rows = kind <= kLoadV ? BKV : (kind == kLoadHbar ? D : kChunk);
+        y = kind <= kLoadV ? j * BKV : (kind == kLoadHbar ? 0 : j * kChunk);
+      };
+      auto load = [&](int kind, int j, int bh) -> bool {
         const int slot = ring % C::NSLOT;
         const uint32_t ph = (ring / C::NSLOT) & 1;
         if (!mbar_wait(&bars.kv_empty[slot], ph ^ 1, abort_flag)) return false;
         unsigned char* dst = sSlot + slot * C::SLOT;
-        const int rows = kind <= 1 ? BKV : (kind == 4 ? D : kChunk);
+        const CUtensorMap* map;
+        int y, rows;
+        tile_map(kind, j, map, y, rows);
         mbar_arrive_expect_tx(&bars.kv_full[slot], rows * D * 2);
-        const CUtensorMap* map = kind == 0 ? &tmK : kind == 1 ? &tmV : kind == 2 ? &tmKb
-                                 : kind == 3 ? &tmVs : &tmHb;
-        const int y = kind <= 1 ? j * BKV : (kind == 4 ? 0 : j * kChunk);
         // one 4-D box: 64 columns x rows x (D/64) column groups; lands as D/64 swizzled
         // [rows x 64] sub-tiles, sub-tile h at byte offset h * rows * 128
         tma_load_4d(dst, map, &bars.kv_full[slot], 0, y, 0, bh);
         ++ring;
-        (void)t_idx;
         return true;
       };
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-        const int bh = item / p.n_qt, qt = item % p.n_qt;
-        const Lists lists = item_lists<C::QBPT>(p, bh, qt);
-        const int n_ex = count_exact<C::QBPT>(lists);
-        const int n = n_ex + n_ch;
-        const int qb = it & 1;
-        if (!mbar_wait(&bars.q_empty[qb], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars.q_full[qb], p.qbox * D * 2);
-        if (p.qbox == kBQ) {
-          tma_load_4d(smem + qb * C::QBYTES, &tmQ, &bars.q_full[qb], 0, qt * kBQ, 0, bh);
-        } else {  // L < 128: one box per column group, at the 128-row sub-tile stride
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + qb * C::QBYTES + h * kBQ * 128, &tmQ, &bars.q_full[qb], 0, 0, h, bh);
-        }
-        ++q_issued;
-        Lists lk = lists, lv = lists;
-        for (int t = 0; t < n && ok; ++t) {
-          if (t < n_ex) ok = load_slot(0, t, lk.next(), bh);
-          else ok = load_slot(2, t, t - n_ex, bh);
-          if (ok && t >= 1) {
-            const int u = t - 1;
-            if (u < n_ex) ok = load_slot(1, u, lv.next(), bh);
-            else ok = load_slot(3, u, u - n_ex, bh);
+      // the loads of one step of stream x, in the MMA issuer's order
+      auto step = [&](StreamPos<C::QBPT>& s, int x) -> bool {
+        if (s.t == 0) {
+          if (s.n == 0) {
+            s.advance(p, x, n_ch);
+            return true;
           }
+          const bool r = s.n_ex > 0 ? load(kLoadK, s.lk.next(), s.bh) : load(kLoadKbar, 0, s.bh);
+          s.t = 1;
+          return r;
         }
-        if (ok && n >= 1) {
-          const int u = n - 1;
-          if (u < n_ex) ok = load_slot(1, u, lv.next(), bh);
-          else ok = load_slot(3, u, u - n_ex, bh);
+        const int u = s.t - 1;
+        if (!(u < s.n_ex ? load(kLoadV, s.lv.next(), s.bh) : load(kLoadVsum, u - s.n_ex, s.bh)))
+          return false;
+        if (s.t < s.n) {
+          const bool r = s.t < s.n_ex ? load(kLoadK, s.lk.next(), s.bh)
+                                      : load(kLoadKbar, s.t - s.n_ex, s.bh);
+          ++s.t;
+          return r;
         }
-        if (ok && p.pisa) ok = load_slot(4, 0, 0, bh);
+        const bool r = p.pisa ? load(kLoadHbar, 0, s.bh) : true;
+        s.advance(p, x, n_ch);
+        return r;
+      };
+      StreamPos<C::QBPT> s0, s1;
+      s0.k = s1.k = 0;
+      s0.tiles = s1.tiles = 0;
+      s0.items = s1.items = 0;
+      s0.start(p, 0, n_ch);
+      s1.start(p, 1, n_ch);
+      while (ok && (s0.active(p) || s1.active(p))) {
+        if (s0.active(p) && !(ok = step(s0, 0))) break;
+        if (s1.active(p) && !(ok = step(s1, 1))) break;
       }
       if (!ok) {
         // drain: wait (bounded, ignoring the abort flag) for copies still in flight
@@ -242,108 +354,113 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                  globaltimer_ns() - t0 < 100000000ull) {
           }
         }
-        for (int r = max(0, q_issued - 2); r < q_issued; ++r) {
-          while (!mbar_try_wait(&bars.q_full[r & 1], (r >> 1) & 1) &&
-                 globaltimer_ns() - t0 < 100000000ull) {
-          }
-        }
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      uint32_t ring = 0, g = 0;
-      int it = 0;
+      uint32_t ring = 0;
       bool ok = true;
       constexpr uint32_t idesc_s_ex = idesc_bf16_f32(kBQ, BKV, false, false);
       constexpr uint32_t idesc_s_ch = idesc_bf16_f32(kBQ, kChunk, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, D, false, true);
-      auto wait_slot = [&](uint32_t& slot_out) -> bool {
+      auto wait_slot = [&](uint32_t& addr) -> bool {
         const int slot = ring % C::NSLOT;
         if (!mbar_wait(&bars.kv_full[slot], (ring / C::NSLOT) & 1, abort_flag)) return false;
         tc_fence_after();
-        slot_out = slot;
+        addr = smem_u32(sSlot + slot * C::SLOT);
         ++ring;
         return true;
       };
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
-        const int bh = item / p.n_qt, qt = item % p.n_qt;
-        const Lists lists = item_lists<C::QBPT>(p, bh, qt);
-        const int n_ex = count_exact<C::QBPT>(lists);
-        const int n = n_ex + n_ch;
-        const int qb = it & 1;
-        if (!mbar_wait(&bars.q_full[qb], (it >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + qb * C::QBYTES);
-        bool o_free_done = (it == 0);
-        auto wait_o_free = [&]() -> bool {
-          if (o_free_done) return true;
-          if (!mbar_wait(&bars.o_free, (it - 1) & 1, abort_flag)) return false;
+      auto release_slot = [&]() { mma_commit(&bars.kv_empty[(ring - 1) % C::NSLOT]); };
+      // S = Q K^T (K-major operands) into the stream's S buffer
+      auto issue_s = [&](int x, uint32_t k_addr, int rows, uint32_t idesc) {
+        const uint32_t q_addr = smem_u32(smem + x * C::QBYTES);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t adesc =
+              smem_desc_sw128(q_addr + (k / 4) * (kBQ * 128) + (k % 4) * 32, 16, 1024);
+          const uint64_t bdesc =
+              smem_desc_sw128(k_addr + (k / 4) * (rows * 128) + (k % 4) * 32, 16, 1024);
+          mma_ss(tmem + C::S_COL(x), adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+        }
+      };
+      // one step of stream x (see StreamPos); false when a wait gave up
+      auto mstep = [&](StreamPos<C::QBPT>& s, const int x) -> bool {
+        if (s.t == 0) {
+          // item start: its Q is loaded and the previous item's epilogue has read
+          // this stream's S (first-order T) and O
+          if (!mbar_wait(&bars.q_full[x], s.items & 1, abort_flag)) return false;
+          if (s.items > 0 && !mbar_wait(&bars.o_free[x], (s.items - 1) & 1, abort_flag))
+            return false;
           tc_fence_after();
-          o_free_done = true;
+          if (s.n == 0) {
+            mma_commit(&bars.o_final[x]);
+            s.advance(p, x, n_ch);
+            return true;
+          }
+          uint32_t k_addr;
+          if (!wait_slot(k_addr)) return false;
+          const bool chunk = 0 >= s.n_ex;
+          issue_s(x, k_addr, chunk ? kChunk : BKV, chunk ? idesc_s_ch : idesc_s_ex);
+          release_slot();
+          mma_commit(&bars.s_full[x]);
+          s.t = 1;
           return true;
-        };
-        auto issue_pv = [&](int u) -> bool {
-          const uint32_t gu = g + u, buf = gu & 1;
-          if (!mbar_wait(&bars.p_full[buf], (gu >> 1) & 1, abort_flag)) return false;
-          tc_fence_after();
-          uint32_t slot;
-          if (!wait_slot(slot)) return false;
-          if (u == 0 && !wait_o_free()) return false;
-          const bool chunk = u >= n_ex;
-          const int kdim = chunk ? kChunk : BKV;
-          const uint32_t v_addr = smem_u32(sSlot + slot * C::SLOT);
+        }
+        // PV(u) with P (bf16, TMEM) of tile u
+        const int u = s.t - 1;
+        if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag)) return false;
+        tc_fence_after();
+        uint32_t v_addr;
+        if (!wait_slot(v_addr)) return false;
+        {
+          const int kdim = u >= s.n_ex ? kChunk : BKV;
           for (int k = 0; k < kdim / 16; ++k) {
             const uint64_t bdesc = smem_desc_sw128(v_addr + k * 2048, kdim * 128, 1024);
-            mma_ts(tmem + C::O_COL, tmem + (buf ? 128u : 0u) + k * 8, bdesc, idesc_o,
+            mma_ts(tmem + C::O_COL(x), tmem + C::S_COL(x) + k * 8, bdesc, idesc_o,
                    (u > 0 || k > 0) ? 1u : 0u);
           }
-          mma_commit(&bars.kv_empty[slot]);
-          mma_commit(&bars.o_bar);
+        }
+        release_slot();
+        if (s.t < s.n) {
+          uint32_t k_addr;
+          if (!wait_slot(k_addr)) return false;
+          const bool chunk = s.t >= s.n_ex;
+          issue_s(x, k_addr, chunk ? kChunk : BKV, chunk ? idesc_s_ch : idesc_s_ex);
+          release_slot();
+          mma_commit(&bars.s_full[x]);
+          ++s.t;
           return true;
-        };
-        for (int t = 0; t < n && ok; ++t) {
-          uint32_t slot;
-          if (!wait_slot(slot)) { ok = false; break; }
-          const bool chunk = t >= n_ex;
-          const int rows = chunk ? kChunk : BKV;
-          const uint32_t buf = (g + t) & 1;
-          const uint32_t k_addr = smem_u32(sSlot + slot * C::SLOT);
+        }
+        if (p.pisa) {
+          // first-order term T = Q Hbar into this stream's (now free) S buffer
+          uint32_t h_addr;
+          if (!wait_slot(h_addr)) return false;
+          const uint32_t q_addr = smem_u32(smem + x * C::QBYTES);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint64_t adesc =
                 smem_desc_sw128(q_addr + (k / 4) * (kBQ * 128) + (k % 4) * 32, 16, 1024);
-            const uint64_t bdesc =
-                smem_desc_sw128(k_addr + (k / 4) * (rows * 128) + (k % 4) * 32, 16, 1024);
-            mma_ss(tmem + (buf ? 128u : 0u), adesc, bdesc, chunk ? idesc_s_ch : idesc_s_ex,
-                   k > 0 ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(h_addr + k * 2048, D * 128, 1024);
+            mma_ss(tmem + C::S_COL(x), adesc, bdesc, idesc_o, k > 0 ? 1u : 0u);
           }
-          mma_commit(&bars.kv_empty[slot]);
-          mma_commit(&bars.s_full[buf]);
-          if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+          release_slot();
         }
-        if (ok && n >= 1) ok = issue_pv(n - 1);
-        if (ok && p.pisa) {
-          uint32_t slot;
-          ok = wait_slot(slot) && wait_o_free();
-          if (ok) {
-            const uint32_t h_addr = smem_u32(sSlot + slot * C::SLOT);
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t adesc =
-                  smem_desc_sw128(q_addr + (k / 4) * (kBQ * 128) + (k % 4) * 32, 16, 1024);
-              const uint64_t bdesc = smem_desc_sw128(h_addr + k * 2048, D * 128, 1024);
-              mma_ss(tmem + C::T_COL, adesc, bdesc, idesc_o, k > 0 ? 1u : 0u);
-            }
-            mma_commit(&bars.kv_empty[slot]);
-          }
-        }
-        if (ok) ok = wait_o_free();
-        if (!ok) break;
-        mma_commit(&bars.q_empty[qb]);
-        mma_commit(&bars.o_final);
-        g += n;
+        mma_commit(&bars.o_final[x]);
+        s.advance(p, x, n_ch);
+        return true;
+      };
+      StreamPos<C::QBPT> s0, s1;
+      s0.k = s1.k = 0;
+      s0.tiles = s1.tiles = 0;
+      s0.items = s1.items = 0;
+      s0.start(p, 0, n_ch);
+      s1.start(p, 1, n_ch);
+      while (ok && (s0.active(p) || s1.active(p))) {
+        if (s0.active(p) && !(ok = mstep(s0, 0))) break;
+        if (s1.active(p) && !(ok = mstep(s1, 1))) break;
       }
       // every issued MMA must complete before TMEM is released
       mma_commit(&bars.done);
@@ -352,15 +469,38 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       }
     }
     __syncwarp();
+  }
   } else {
-    // ============================================================ softmax + epilogue
+    setmaxnreg_inc<kRegsSoftmax>();
+    // ==================================================== softmax + epilogue (per stream)
+    const int x = warp / 4;                    // stream of this warpgroup
     const int quad = warp % 4;                 // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;          // query row within the tile
+    const bool q_loader = quad == 0 && lane == 0;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    uint32_t g = 0, pv = 0;
-    int it = 0;
+    const uint32_t s_base = tmem + lane_addr + C::S_COL(x);
+    const uint32_t o_base = tmem + lane_addr + C::O_COL(x);
+    unsigned char* sq = smem + x * C::QBYTES;
+    auto load_q = [&](int item) {
+      const int bh = item / p.n_qt, qt = item % p.n_qt;
+      mbar_arrive_expect_tx(&bars.q_full[x], p.qbox * D * 2);
+      if (p.qbox == kBQ) {
+        tma_load_4d(sq, &tmQ, &bars.q_full[x], 0, qt * kBQ, 0, bh);
+      } else {  // L < 128: one box per column group, at the 128-row sub-tile stride
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_4d(sq + h * kBQ * 128, &tmQ, &bars.q_full[x], 0, 0, h, bh);
+      }
+    };
+    int q_issued = 0;
+    if (q_loader && stream_item(0, x) < p.n_items) {
+      load_q(stream_item(0, x));
+      q_issued = 1;
+    }
+    uint32_t tiles = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++it) {
+    for (int k = 0; stream_item(k, x) < p.n_items && ok; ++k) {
+      const int item = stream_item(k, x);
       const int bh = item / p.n_qt, qt = item % p.n_qt;
       Lists lists = item_lists<C::QBPT>(p, bh, qt);
       const int n_ex = count_exact<C::QBPT>(lists);
@@ -375,42 +515,23 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       float m_run = -INFINITY, l = 0.f, sa = 0.f;
 
       for (int t = 0; t < n; ++t) {
-        const uint32_t gt = g + t, buf = gt & 1;
-        ok = mbar_wait(&bars.s_full[buf], (gt >> 1) & 1, abort_flag);
+        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
         const bool chunk = t >= n_ex;
-        const uint32_t s_addr = tmem + lane_addr + (buf ? 128u : 0u);
-        float s[128];
-        {
-          uint32_t r[32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if (c * 32 < (chunk ? kChunk : BKV)) {
-              tmem_ld32(s_addr + c * 32, r);
-#pragma unroll
-              for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
-            }
-          }
-          tmem_wait_ld();
-        }
-        // tile width: 128 for centroid chunks, BKV for exact tiles (compile-time for 128)
-        const int N = BKV == kChunk ? kChunk : (chunk ? kChunk : BKV);
+        bool skip = false;          // whole tile masked for this row
+        uint32_t excl[4] = {0u, 0u, 0u, 0u};
         if (!chunk) {
           if (C::QBPT == 2) {
             const int j = lists.next();
             const bool member = mp < me && __ldg(p.col_idx + mp) == j;
             if (member) ++mp;
-            if (!member) {
-#pragma unroll
-              for (int x = 0; x < BKV; ++x) s[x] = -INFINITY;
-            }
+            skip = !member;
           }
         } else {
-          // centroid chunk: mask selected blocks and indices past M
+          // centroid chunk: exclude the selected blocks and indices past M
           const int base = (t - n_ex) * kChunk;
-          uint32_t excl[4] = {0u, 0u, 0u, 0u};
           while (cp < me) {
             const int cj = __ldg(p.col_idx + cp);
             if (cj >= base + kChunk) break;
@@ -419,41 +540,47 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           }
           const int valid = has_blk ? min(kChunk, p.M - base) : 0;
 #pragma unroll
-          for (int x = 0; x < kChunk; ++x)
-            if (x >= valid || ((excl[x >> 5] >> (x & 31)) & 1u)) s[x] = -INFINITY;
-        }
-        // row max (log2 domain); 8 independent chains keep the FMNMX latency hidden
-        float mxa[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) mxa[a] = s[a];
-#pragma unroll
-        for (int x = 8; x < 128; x += 8) {
-          if (x < N) {
-#pragma unroll
-            for (int a = 0; a < 8; ++a) mxa[a] = fmaxf(mxa[a], s[x + a]);
+          for (int w = 0; w < 4; ++w) {
+            const int lo = w * 32;
+            if (valid <= lo) excl[w] = 0xffffffffu;
+            else if (valid < lo + 32) excl[w] |= 0xffffffffu << (valid - lo);
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                               fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
-                         p.scale_log2;
+        // pass 1: this thread's whole S row into registers (one wait), the excluded
+        // entries of a centroid chunk set to -inf, then the row max
+        const int cols = chunk ? kChunk : BKV;
+        uint32_t r[128];
+        float mx = -INFINITY;
+        if (!skip) {
+          tmem_ld32(s_base, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(s_base + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+          if (cols == 128) {
+            tmem_ld32(s_base + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+            tmem_ld32(s_base + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+          }
+          tmem_wait_ld();
+          if (chunk) {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              if ((excl[e >> 5] >> (e & 31)) & 1u) r[e] = __float_as_uint(-INFINITY);
+          }
+          mx = cols == 128 ? row_max<128>(r) : row_max<64>(r);
+        }
+        mx *= p.scale_log2;
         const bool need = mx > m_run + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mx : m_run;
           const float factor = need ? ex2(m_run - m_new) : 1.0f;
           if (t > 0) {
-            ok = mbar_wait(&bars.o_bar, (pv + t - 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t o_addr = tmem + lane_addr + C::O_COL;
+            // PV(t-1) was issued before S(t), so it has completed: rescale O in TMEM
 #pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
-              uint32_t r[32];
-              tmem_ld32(o_addr + c, r);
+            for (int c = 0; c < D; c += 16) {
+              uint32_t ro[16];
+              tmem_ld16(o_base + c, ro);
               tmem_wait_ld();
 #pragma unroll
-              for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * factor);
-              tmem_st32(o_addr + c, r);
+              for (int e = 0; e < 16; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * factor);
+              tmem_st16(o_base + c, ro);
             }
             tmem_wait_st();
           }
@@ -462,26 +589,20 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           m_run = m_new;
         }
         const float m_ref = m_run == -INFINITY ? 0.f : m_run;
-        // P = 2^(s*scale_log2 - m) as bf16 pairs, written back over the first N/2
-        // columns of this S buffer one 64-column half at a time (all S values are
-        // already in registers, so the overwrite is safe)
-        const uint32_t p_addr = tmem + lane_addr + (buf ? 128u : 0u);
-        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // pass 2: P = 2^(s*scale_log2 - m) as bf16 pairs over the first cols/2 columns of
+        // the S buffer (the row is in registers, so the overwrite is safe)
+        float rs = 0.f;
+        if (skip) {
+          uint32_t z[32];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          if (hf * 64 < N) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int x = 0; x < 64; x += 2) {
-              const float e0 = ex2(fmaf(s[hf * 64 + x], p.scale_log2, -m_ref));
-              const float e1 = ex2(fmaf(s[hf * 64 + x + 1], p.scale_log2, -m_ref));
-              sm[(x / 2) & 7] += e0 + e1;
-              pk[x / 2] = pack_bf16x2(e0, e1);
-            }
-            tmem_st32(p_addr + hf * 32, pk);
-          }
+          for (int e = 0; e < 32; ++e) z[e] = 0u;
+          tmem_st32(s_base, z);
+          if (cols == 128) tmem_st32(s_base + 32, z);
+        } else if (chunk) {
+          rs = row_exp<128, false>(r, p.scale_log2, m_ref, s_base);
+        } else {
+          rs = row_exp<BKV, true>(r, p.scale_log2, m_ref, s_base);
         }
-        const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
         if (chunk) {
           l += (float)BKV * rs;
           sa += rs;
@@ -490,63 +611,72 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars.p_full[buf]);
+        mbar_arrive(&bars.p_full[x]);
       }
       if (!ok) break;
 
       // ---------------------------------------------------------------- epilogue
-      ok = mbar_wait(&bars.o_final, it & 1, abort_flag);
+      ok = mbar_wait(&bars.o_final[x], k & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      // every MMA of this item has completed: Q's buffer is free for the next item
+      if (q_loader && stream_item(k + 1, x) < p.n_items) {
+        load_q(stream_item(k + 1, x));
+        ++q_issued;
+      }
       const bool write = row_g < p.L;
       __nv_bfloat16* orow = p.O + ((size_t)bh * p.L + (write ? row_g : 0)) * D;
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
       const float c1 = p.scale * sa;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t ro[32], rt[32];
+      for (int c = 0; c < D; c += 16) {
+        uint32_t ro[16], rt[16];
         if (n > 0) {
-          tmem_ld32(tmem + lane_addr + C::O_COL + c, ro);
-          if (p.pisa) tmem_ld32(tmem + lane_addr + C::T_COL + c, rt);
+          tmem_ld16(o_base + c, ro);
+          if (p.pisa) tmem_ld16(s_base + c, rt);  // T = Q Hbar sits in the S buffer
           tmem_wait_ld();
         }
-        uint32_t packed[16];
+        uint32_t packed[8];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
+        for (int e = 0; e < 16; e += 2) {
           float a0 = 0.f, a1 = 0.f;
           if (n > 0) {
-            a0 = __uint_as_float(ro[x]);
-            a1 = __uint_as_float(ro[x + 1]);
+            a0 = __uint_as_float(ro[e]);
+            a1 = __uint_as_float(ro[e + 1]);
             if (p.pisa) {
-              a0 = fmaf(c1, __uint_as_float(rt[x]), a0);
-              a1 = fmaf(c1, __uint_as_float(rt[x + 1]), a1);
+              a0 = fmaf(c1, __uint_as_float(rt[e]), a0);
+              a1 = fmaf(c1, __uint_as_float(rt[e + 1]), a1);
             }
           }
-          packed[x / 2] = pack_bf16x2(a0 * inv_l, a1 * inv_l);
+          packed[e / 2] = pack_bf16x2(a0 * inv_l, a1 * inv_l);
         }
         if (write) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
-                                packed[4 * v + 3]);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
       }
       if (write && p.lse)
         p.lse[(size_t)bh * p.L + row_g] =
             l > 0.f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
-      mbar_arrive(&bars.o_free);
-      g += n;
-      pv += n;
+      mbar_arrive(&bars.o_free[x]);
+      tiles += n;
+    }
+    if (!ok && q_loader && q_issued > 0) {
+      // drain this stream's last Q copy (bounded) before the CTA exits
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&bars.q_full[x], (q_issued - 1) & 1) &&
+             globaltimer_ns() - t0 < 100000000ull) {
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && abort_sh) report(p.status, BSA_ERR_TIMEOUT);
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -665,6 +795,13 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   cudaError_t e = cudaFuncSetAttribute(k_forward<D, BKV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
+  // setmaxnreg.inc waits until the warpgroups that shrink have released enough registers:
+  // the split must fit in what the launch allocates, or the kernel would never start
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k_forward<D, BKV>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * kRegsControl + 128 * kStreams * kRegsSoftmax)
+    return cudaErrorInvalidConfiguration;
   const int grid = min(p.n_items, sm_count());
   k_forward<D, BKV><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, p);
   return cudaGetLastError();

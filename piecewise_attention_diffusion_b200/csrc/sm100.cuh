@@ -246,6 +246,75 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Warpgroup register reallocation: every warp of the warpgroup executes the same call.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes, each rounded
+// to nearest like its scalar form).
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_from(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+
+// Coefficients c0..c3 of the degree-3 polynomial for 2^f on [-1/2, 1/2] that minimises
+// the maximum relative error (7.5e-5), from the Remez fit in exp2_poly_fit.py.
+constexpr float kEx2C0 = 0.99992806f, kEx2C1 = 0.69326097f, kEx2C2 = 0.24261113f,
+                kEx2C3 = 0.05517167f;
+
+// 2^x for a pair, on the FMA pipe, for x <= 8 (larger x are not produced by the callers).
+// Cody-Waite style split x = n + f: n = rint(x) by adding 1.5 * 2^23 (the sum's low
+// mantissa bits then hold n), f = x - n in [-1/2, 1/2]; 2^f from the polynomial; n is
+// added to the exponent field. The sum's bits are 0x4B400000 + n and the constant's set
+// bits all sit at or above bit 22, so shifting them left by 23 leaves n << 23 (mod 2^32).
+// Inputs below -126 are clamped to -126: the result there is a tiny positive number.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = add2(x, make_float2(kShift, kShift));
+  const float2 f = sub2(x, sub2(t, make_float2(kShift, kShift)));
+  float2 q = fma2(f, make_float2(kEx2C3, kEx2C3), make_float2(kEx2C2, kEx2C2));
+  q = fma2(q, f, make_float2(kEx2C1, kEx2C1));
+  q = fma2(q, f, make_float2(kEx2C0, kEx2C0));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Pack two fp32 into bf16x2 (round to nearest even): `lo` in the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
