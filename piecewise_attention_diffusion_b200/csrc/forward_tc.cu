@@ -511,33 +511,35 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int32_t* rp = p.csr_per_head ? p.row_ptr + (size_t)bh * (p.M + 1) : p.row_ptr;
       const int mb = has_blk ? __ldg(rp + iq) : 0;
       const int me = has_blk ? __ldg(rp + iq + 1) : 0;
-      int mp = mb, cp = mb;
+      int mp = mb;
       float m_run = -INFINITY, l = 0.f, sa = 0.f;
 
       for (int t = 0; t < n; ++t) {
-        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
         const bool chunk = t >= n_ex;
-        bool skip = false;          // whole tile masked for this row
         uint32_t excl[4] = {0u, 0u, 0u, 0u};
-        if (!chunk) {
-          if (C::QBPT == 2) {
-            const int j = lists.next();
-            const bool member = mp < me && __ldg(p.col_idx + mp) == j;
-            if (member) ++mp;
-            skip = !member;
-          }
-        } else {
-          // centroid chunk: exclude the selected blocks and indices past M
+        if (chunk) {
+          // centroid chunk: exclude this row's selected blocks and the indices past M.
+          // The 32 rows of a warp share one query block, so the lanes read its list
+          // together (coalesced) and OR their bits across the warp; this runs before the
+          // wait for S, which hides the loads' latency
           const int base = (t - n_ex) * kChunk;
-          while (cp < me) {
-            const int cj = __ldg(p.col_idx + cp);
-            if (cj >= base + kChunk) break;
-            if (cj >= base) excl[(cj - base) >> 5] |= 1u << ((cj - base) & 31);
-            ++cp;
+          uint32_t w0 = 0u, w1 = 0u, w2 = 0u, w3 = 0u;
+          for (int e0 = mb; e0 < me; e0 += 32) {
+            const int e = e0 + lane;
+            const int cj = e < me ? __ldg(p.col_idx + e) - base : -1;
+            if (cj >= 0 && cj < kChunk) {
+              const uint32_t bit = 1u << (cj & 31);
+              const int wd = cj >> 5;
+              w0 |= wd == 0 ? bit : 0u;
+              w1 |= wd == 1 ? bit : 0u;
+              w2 |= wd == 2 ? bit : 0u;
+              w3 |= wd == 3 ? bit : 0u;
+            }
           }
+          excl[0] = __reduce_or_sync(0xffffffffu, w0);
+          excl[1] = __reduce_or_sync(0xffffffffu, w1);
+          excl[2] = __reduce_or_sync(0xffffffffu, w2);
+          excl[3] = __reduce_or_sync(0xffffffffu, w3);
           const int valid = has_blk ? min(kChunk, p.M - base) : 0;
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
@@ -545,6 +547,17 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (valid <= lo) excl[w] = 0xffffffffu;
             else if (valid < lo + 32) excl[w] |= 0xffffffffu << (valid - lo);
           }
+        }
+        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        bool skip = false;          // whole tile masked for this row
+        if (!chunk && C::QBPT == 2) {
+          const int j = lists.next();
+          const bool member = mp < me && __ldg(p.col_idx + mp) == j;
+          if (member) ++mp;
+          skip = !member;
         }
         // pass 1: this thread's whole S row into registers (one wait), the excluded
         // entries of a centroid chunk set to -inf, then the row max

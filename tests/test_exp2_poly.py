@@ -10,7 +10,7 @@ from piecewise_attention_diffusion_b200 import exp2_poly_fit
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
                    "piecewise_attention_diffusion_b200", "csrc", "sm100.cuh")
-BOUND = 8e-5  # relative; bf16 keeps 8 significant bits (half ulp 2^-9 ~ 2e-3)
+BOUND = 8e-5  # relative; far below bf16's unit roundoff 2^-8 ~ 3.9e-3
 
 
 def _kernel_constants():
@@ -48,15 +48,15 @@ def test_constants_match_the_fit():
 
 
 def test_relative_error_bound_over_the_used_range():
-    x = np.concatenate([np.linspace(-126.0, 8.0, 2_000_001),
-                        np.random.default_rng(0).uniform(-30, 8, 1_000_000)]).astype(np.float32)
+    x = np.concatenate([np.linspace(-126.0, 16.0, 2_000_001),
+                        np.random.default_rng(0).uniform(-30, 16, 1_000_000)]).astype(np.float32)
     got = _ex2_poly(x).astype(np.float64)
     want = np.exp2(x.astype(np.float64))
     normal = want >= 2.0 ** -125
     rel = np.abs(got[normal] - want[normal]) / want[normal]
     assert rel.max() < BOUND
     # integers are exact up to the polynomial's value at 0
-    xi = np.arange(-120, 9).astype(np.float32)
+    xi = np.arange(-120, 17).astype(np.float32)
     np.testing.assert_allclose(_ex2_poly(xi), np.exp2(xi.astype(np.float64)), rtol=1e-4)
     # below the clamp the result is a tiny positive number, never negative or NaN
     tiny = _ex2_poly(np.asarray([-1e30, -200.0, -126.7], dtype=np.float32))

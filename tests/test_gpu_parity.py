@@ -15,7 +15,7 @@ import torch
 import oracle as orc
 from piecewise_attention_diffusion_b200 import bsattn as b
 from piecewise_attention_diffusion_b200 import synth
-from tests._util import (assert_close_out, f64, rel_l2, rows_agree_up_to_ties)
+from tests._util import (REL_L2_TOL, assert_close_out, f64, rel_l2, rows_agree_up_to_ties)
 
 pytestmark = pytest.mark.gpu
 
@@ -214,6 +214,56 @@ def test_forward_shapes_and_ragged_tiles(L, block, d, kk, mode):
     kbar, vsum, Hbar, Mn = _oracle_stats(k, v, block)
     rp, ci, _ = orc.route(f64(q), kbar, Mn, block, kk, 1.0, 1 / math.sqrt(d))
     _forward_check(w, q, k, v, rp, ci, 1, mode, (kbar, vsum, Hbar))
+
+
+@pytest.mark.parametrize("mode", [b.MODE_KEEP_OR_DROP, b.MODE_PISA])
+def test_forward_growing_scores_exercise_the_rescale(mode):
+    """Key block j is scaled by 1 + 2.5 j and every query block selects the even blocks,
+    so each exact tile raises the row max by ~20 in the log2 domain: the kernel's lazy O
+    rescale (threshold 2^8) fires on every tile, and in PISA mode also on the centroid
+    sweep over the odd blocks.
+
+    The attention is then nearly one-hot and |O| reaches ~4.6, where rounding the output
+    to bf16 alone (unit roundoff 2^-8) can move it by up to 0.018: the fixed max-abs bound
+    of the workload configs (whose outputs average many rows and stay small) does not
+    apply. The bound here is derived instead: output rounding 2^-8 |o|, plus the bf16
+    rounding of P, which moves o = sum_i w_i v_i by at most 2^-8 sum_i w_i |v_i| <=
+    2^-8 max |v|, plus 1e-3 for fp32 accumulation."""
+    w = synth.Workload("grow", 1, 2, 2048, 128, 128, "pisa", k_top=8, generator="iid")
+    q, k, v = synth.make_qkv(w, seed=11)
+    M = w.n_blocks
+    scale_j = torch.repeat_interleave(1.0 + 2.5 * torch.arange(M, dtype=torch.float32), w.block)
+    k = (k.float() * scale_j[None, None, :, None]).to(k.dtype)
+    rp = np.arange(0, M * 8 + 1, 8, dtype=np.int32)
+    ci = np.tile(np.arange(0, M, 2, dtype=np.int32), M)
+    kbar, vsum, Hbar, Mn = _oracle_stats(k, v, w.block)
+    grp, gci = _csr_to_gpu(rp, ci)
+    st = _status()
+    stats = _stats_to_gpu(kbar, vsum, Hbar) if mode == b.MODE_PISA else None
+    O, lse = b.forward(q.to(DEV), k.to(DEV), v.to(DEV), w.block, grp, gci, 0, mode,
+                       stats=stats, want_lse=True, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    scale = 1 / math.sqrt(w.head_dim)
+    for h in range(2):
+        qf, kf, vf = (f64(x[0, h]) for x in (q, k, v))
+        hrp, hci = orc.head_csr(rp, ci, h, M, 0)
+        if mode == b.MODE_PISA:
+            want, wl = orc.pisa_head(qf, kf, vf, hrp, hci, w.block, scale, kbar[h], vsum[h],
+                                     Hbar[h])
+        else:
+            want, wl = orc.keep_or_drop_head(qf, kf, vf, hrp, hci, w.block, scale)
+        got = f64(O[0, h])
+        assert np.isfinite(got).all()
+        tol = 1e-3 + 2.0 ** -8 * (np.abs(want) + np.abs(vf).max())
+        assert (np.abs(got - want) <= tol).all(), float((np.abs(got - want) - tol).max())
+        assert rel_l2(got, want) <= REL_L2_TOL
+        ltol = np.full(w.seq_len, 2e-3)
+        if mode == b.MODE_PISA:  # centroid scores from bf16 kbar (see _forward_check)
+            ltol += (scale * np.abs(qf) @ np.abs(kbar[h]).T * 2.0 ** -8).max(axis=1)
+        assert (np.abs(f64(lse[h]) - wl) <= ltol).all()
+        print(f"[parity] grow mode={mode} head {h} max-abs {np.abs(got - want).max():.2e} "
+              f"rel-L2 {rel_l2(got, want):.2e}")
 
 
 def test_forward_full_density_pisa_equals_keep_or_drop_equals_dense():
