@@ -36,14 +36,28 @@ LAMBDA = 1.0
 
 
 # ------------------------------------------------------------------ FLOP counting
-def forward_flops(w, k_top: int, mode: str) -> float:
-    """Executed FLOPs of bsa_forward: per (batch, head, query block)
-    k * 4 B^2 d  (+ PISA: B * (4 d |U_i| + 2 d^2)); exps and softmax not counted."""
+def forward_flops(w, k_top: int, mode: str, row_lens=None) -> float:
+    """Executed FLOPs of bsa_forward: per (batch, head, query block i)
+    |S_i| * 4 B^2 d  (+ PISA: B * (4 d |U_i| + 2 d^2)); exps and softmax not counted.
+    |S_i| = k_top for routed lists, the row length for a fixed mask (row_lens)."""
     M, B, d = w.n_blocks, w.block, w.head_dim
-    per_qb = k_top * 4.0 * B * B * d
-    if mode == "pisa":
-        per_qb += B * (4.0 * d * (M - k_top) + 2.0 * d * d)
-    return w.batch * w.heads * M * per_qb
+    lens = [k_top] * M if row_lens is None else list(row_lens)
+    total = 0.0
+    for n in lens:
+        total += n * 4.0 * B * B * d
+        if mode == "pisa":
+            total += B * (4.0 * d * (M - n) + 2.0 * d * d)
+    return w.batch * w.heads * total
+
+
+def launches_per_step(w) -> int:
+    """Kernels one step launches: precompute 3 (statistics, reduce, norm; skipped for a
+    fixed keep-or-drop mask), route 1 (not for a fixed mask), forward: list validation,
+    the PISA statistics' bf16 conversion, the forward kernel."""
+    pre = 0 if (w.mask and w.mode != "pisa") else 3
+    route = 0 if w.mask else 1
+    fwd = 3 if w.mode == "pisa" else 2
+    return pre + route + fwd
 
 
 def precompute_flops(w) -> float:
@@ -203,11 +217,18 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
     heads = list(range(heads_sample))
     q, k, v = synth.make_qkv(w, seed=seed, heads=heads)
     scale = 1 / math.sqrt(w.head_dim)
+    fixed = orc.dense_to_csr(orc.mask_dense(**w.mask)) if w.mask else None
     t0 = time.perf_counter()
     for h in heads:
         qf, kf, vf = (x[h].to(torch.float64).numpy() for x in (q, k, v))
+        if fixed is not None and w.mode != "pisa":
+            orc.keep_or_drop_head(qf, kf, vf, fixed[0], fixed[1], w.block, scale)
+            continue
         kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block)
-        rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale)
+        if fixed is not None:
+            rp, ci = fixed
+        else:
+            rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale)
         if w.mode == "pisa":
             orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar)
         else:
@@ -215,8 +236,10 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
     dt = time.perf_counter() - t0
     BH = w.batch * w.heads
     return {"seconds_sample": dt, "seconds_full_est": dt * BH / len(heads), "cores": threads,
-            "sample": f"{len(heads)} of {BH} heads, each fully precomputed, routed and "
-                      f"attended (all {w.n_blocks} query blocks); time scaled by heads"}
+            "sample": f"{len(heads)} of {BH} heads, each fully "
+                      f"{'precomputed and ' if (w.mode == 'pisa' or not w.mask) else ''}"
+                      f"{'' if w.mask else 'routed and '}attended (all {w.n_blocks} query "
+                      f"blocks{', fixed mask' if w.mask else ''}); time scaled by heads"}
 
 
 # --------------------------------------------------------------------- our arm
@@ -225,7 +248,7 @@ def run_ours(args, w, world, rank, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    k_top = w.top_k()
+    k_top = 0 if w.mask else w.top_k()  # a fixed mask has no top-k
     BH, M, L, d = w.batch * w.heads, w.n_blocks, w.seq_len, w.head_dim
     q, k, v = synth.make_qkv(w, seed=args.seed + rank)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -233,8 +256,18 @@ def run_ours(args, w, world, rank, local):
     f32 = dict(dtype=torch.float32, device=dev)
     stats = dict(kbar=torch.empty(BH, M, d, **f32), vsum=torch.empty(BH, M, d, **f32),
                  Hbar=torch.empty(BH, d, d, **f32), Mnorm=torch.empty(BH, M, **f32))
-    rp = torch.empty(BH * (M + 1), dtype=torch.int32, device=dev)
-    ci = torch.empty(BH * M * k_top, dtype=torch.int32, device=dev)
+    if w.mask:
+        # fixed multimodal pattern: one shared list for every head, built once
+        desc = b.MaskDesc(**w.mask)
+        rp, ci = b.build_mask(desc, device=dev, status=st)
+        torch.cuda.synchronize()
+        row_lens = np.diff(rp.cpu().numpy()).tolist()
+        per_head = 0
+    else:
+        rp = torch.empty(BH * (M + 1), dtype=torch.int32, device=dev)
+        ci = torch.empty(BH * M * k_top, dtype=torch.int32, device=dev)
+        row_lens = None
+        per_head = 1
     O = torch.empty_like(qd)
     ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
     ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
@@ -244,16 +277,18 @@ def run_ours(args, w, world, rank, local):
     def step(qx, kx, vx, ev=None):
         if ev:
             ev[0].record(stream)
-        b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
-                         stats["Mnorm"], None, ws_p, st)
+        if not (w.mask and mode != b.MODE_PISA):
+            b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
+                             stats["Mnorm"], None, ws_p, st)
         if ev:
             ev[1].record(stream)
-        b.bsa_route(qx, stats["kbar"], stats["Mnorm"], w.block, k_top, LAMBDA, 0.0, rp, ci,
-                    None, st)
+        if not w.mask:
+            b.bsa_route(qx, stats["kbar"], stats["Mnorm"], w.block, k_top, LAMBDA, 0.0, rp, ci,
+                        None, st)
         if ev:
             ev[2].record(stream)
-        b.bsa_forward(qx, kx, vx, w.block, rp, ci, 1, mode, stats["kbar"], stats["vsum"],
-                      stats["Hbar"], 0.0, O, None, ws_f, st)
+        b.bsa_forward(qx, kx, vx, w.block, rp, ci, per_head, mode, stats["kbar"],
+                      stats["vsum"], stats["Hbar"], 0.0, O, None, ws_f, st)
         if ev:
             ev[3].record(stream)
 
@@ -286,8 +321,9 @@ def run_ours(args, w, world, rank, local):
     if st.item() != 0:
         raise RuntimeError(f"device status {b.status_string(st.item())}")
 
-    F_fwd = forward_flops(w, k_top, w.mode)
-    F_step = F_fwd + precompute_flops(w) + route_flops(w)
+    F_fwd = forward_flops(w, k_top, w.mode, row_lens)
+    F_step = F_fwd + (0.0 if (w.mask and w.mode != "pisa") else precompute_flops(w)) \
+        + (0.0 if w.mask else route_flops(w))
     value = world * F_step / (ms_step * 1e-3) / 1e12
     pk = peaks()
     achieved = F_fwd / (fwd_ms * 1e-3) / 1e12
@@ -332,7 +368,9 @@ def run_ours(args, w, world, rank, local):
         "data": "synthetic (seeded: Q ~ N(0,1); K, V = smooth 3-D field + 0.3 N(0,1))",
         "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": L,
                    "head_dim": d, "block": w.block, "mode": w.mode, "density": w.density,
-                   "k_top": k_top, "lambda": LAMBDA, "parallelism": f"replicas x{world}",
+                   "k_top": None if w.mask else k_top, "lambda": LAMBDA,
+                   "lists": "fixed multimodal mask (shared)" if w.mask else "bsa_route top-k",
+                   "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB)"},
         "forward_ms": round(fwd_ms, 4), "forward_tflops": round(achieved, 3),
         "precompute_ms": round(pre_ms, 4), "route_ms": round(route_ms, 4),
@@ -345,7 +383,7 @@ def run_ours(args, w, world, rank, local):
                      "traffic": load_traffic(w),
                      "algorithmic_bytes": forward_bytes(w, w.mode)},
         "clocks": clocks,
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": launches_per_step(w) * args.steps,
     }
     if e2e:
         line["e2e"] = e2e
@@ -361,8 +399,15 @@ def run_ours(args, w, world, rank, local):
 # --------------------------------------------------------------- reference arm
 def run_reference(args, w, world, rank):
     """The fp64 oracle, as it stands, on the host cores: each step a bounded sample."""
-    k_top = w.top_k()
-    F_step = forward_flops(w, k_top, w.mode) + precompute_flops(w) + route_flops(w)
+    k_top = 0 if w.mask else w.top_k()  # a fixed mask has no top-k
+    row_lens = None
+    if w.mask:
+        import oracle as orc
+        rp, _ = orc.dense_to_csr(orc.mask_dense(**w.mask))
+        row_lens = np.diff(rp).tolist()
+    F_step = forward_flops(w, k_top, w.mode, row_lens) \
+        + (0.0 if (w.mask and w.mode != "pisa") else precompute_flops(w)) \
+        + (0.0 if w.mask else route_flops(w))
     for _ in range(args.warmup):
         oracle_sample(w, k_top, 1, args.seed)
     times, info = [], None

@@ -64,12 +64,13 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   // 1. pooled query of block i: lanes 0..CPR-1 take row r, the next CPR lanes row r+1...
   constexpr int CPR = D / 8;          // 16-byte chunks per row
   constexpr int RPI = 32 / CPR;       // rows per warp iteration
+  constexpr int kUnrollQ = B / RPI >= 32 ? 16 : 8;  // loads in flight per lane
   float* qbar = s_q + warp * D;
   if (active) {
     const __nv_bfloat16* qb = Q + ((size_t)bh * L + (size_t)i * B) * D;
     const int cc = lane % CPR, r0 = lane / CPR;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
+#pragma unroll kUnrollQ
     for (int r = r0; r < B; r += RPI) {
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(qb + (size_t)r * D) + cc);
       float f[8];
@@ -91,12 +92,30 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   // 2. block scores a_j = scale * qbar . kbar_j, centroids staged 64 at a time
   const float* kb = kbar + (size_t)bh * M * D;
   float* sc = s_sc + warp * M;
+  // 16-byte loads when the caller's kbar allows them (each head's slice then does too,
+  // since M * D * 4 is a multiple of 16); unrolled so that a thread's loads are in flight
+  // together rather than one L2 round trip after another
+  const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
   for (int c0 = 0; c0 < M; c0 += kChunkC) {
     const int nc = min(kChunkC, M - c0);
     __syncthreads();
-    for (int e = threadIdx.x; e < nc * D; e += kThreads) {
-      const int r = e / D, c = e % D;
-      s_kb[r * (D + 1) + c] = __ldg(kb + (size_t)(c0 + r) * D + c);
+    if (vec) {
+      const float4* src = reinterpret_cast<const float4*>(kb + (size_t)c0 * D);
+#pragma unroll 8
+      for (int e4 = threadIdx.x; e4 < nc * D / 4; e4 += kThreads) {
+        const float4 v = __ldg(src + e4);
+        float* dst = s_kb + (e4 * 4 / D) * (D + 1) + (e4 * 4 % D);
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
+      }
+    } else {
+#pragma unroll 8
+      for (int e = threadIdx.x; e < nc * D; e += kThreads) {
+        const int r = e / D, c = e % D;
+        s_kb[r * (D + 1) + c] = __ldg(kb + (size_t)(c0 + r) * D + c);
+      }
     }
     __syncthreads();
     if (active) {

@@ -12,12 +12,14 @@ Workloads (sizes named after what they are):
   * tiny_pisa          batch 1, 2 heads, L=512, d=64, block 64
   * multimodal_dit     batch 8, 16 heads, L=1152 (77 text tokens padded to 128 +
                        32x32 image patches), d=64, block 64
+  * multimodal_pisa    the same shape and fixed mask as the exact set of PISA
   * image_pisa         batch 1, 24 heads, L=4096 (64x64 latent), d=128, block 128
   * video_pisa         batch 1, 40 heads, L=16384 (16 frames x 32x32), d=128, block 128
   * sweep_L{L}         batch 1, 24 heads, L in {4096..32768}, d=128, block 128
 """
 from __future__ import annotations
 
+import dataclasses
 import math
 from dataclasses import dataclass, field
 
@@ -61,6 +63,10 @@ def workloads() -> dict:
         "multimodal_dit", 8, 16, 1152, 64, 64, "keep_or_drop", generator="iid",
         mask=dict(n_text_blocks=2, grid_h=4, grid_w=4, radius=1, global_stride=16,
                   global_rows_full=0))
+    # the same fixed pattern as the selection of PISA: the blocks it drops enter through
+    # the Taylor tail (zeroth order per block, first order through Hbar)
+    w["multimodal_pisa"] = dataclasses.replace(w["multimodal_dit"], name="multimodal_pisa",
+                                               mode="pisa")
     w["image_pisa"] = Workload("image_pisa", 1, 24, 4096, 128, 128, "pisa", density=0.15,
                                generator="field2d_hot", grid=(64, 64))
     w["video_pisa"] = Workload("video_pisa", 1, 40, 16384, 128, 128, "pisa", density=0.125,

@@ -204,6 +204,25 @@ def test_forward_multimodal_fixed_mask_keep_or_drop():
                    heads_idx=[0, 17, 63, 127])
 
 
+def test_forward_pisa_over_the_multimodal_fixed_mask():
+    """PISA with S_i from the fixed multimodal pattern (one shared CSR list for every
+    head) and U_i its complement: the blocks the mask drops enter through the Taylor tail
+    instead of vanishing. The forward gets the oracle statistics, so the check isolates it."""
+    w = synth.workloads()["multimodal_dit"]
+    q, k, v = synth.make_qkv(w)
+    keep = orc.mask_dense(**w.mask)
+    rp, ci = orc.dense_to_csr(keep)
+    heads = [0, 17, 63, 127]
+    BH = w.batch * w.heads
+    kf = f64(k).reshape(BH, w.seq_len, w.head_dim)
+    vf = f64(v).reshape(BH, w.seq_len, w.head_dim)
+    stats = [orc.precompute_head(kf[h], vf[h], w.block) for h in range(BH)]
+    kbar = np.stack([s_[0] for s_ in stats])
+    vsum = np.stack([s_[1] for s_ in stats])
+    Hbar = np.stack([s_[3] for s_ in stats])
+    _forward_check(w, q, k, v, rp, ci, 0, b.MODE_PISA, (kbar, vsum, Hbar), heads_idx=heads)
+
+
 @pytest.mark.parametrize("L,block,d,kk", [(576, 64, 64, 3), (640, 128, 128, 2), (64, 64, 128, 1),
                                           (128, 128, 128, 1), (64, 64, 64, 1),
                                           (1152, 64, 128, 5), (768, 128, 64, 6)])
