@@ -66,7 +66,8 @@ typedef enum {
 
 typedef enum {
   BSA_MODE_KEEP_OR_DROP = 0, /* [BSA] §3.3: softmax over the selected blocks only      */
-  BSA_MODE_PISA = 1          /* [PISA] §2: exact S_i + Taylor-approximated U_i         */
+  BSA_MODE_PISA = 1,         /* [PISA] §2: exact S_i + Taylor-approximated U_i         */
+  BSA_MODE_PISA_BLOCK = 2    /* [PISA] §2, first order with each block's own H_j       */
 } bsa_mode;
 
 typedef enum {
@@ -167,6 +168,16 @@ BSA_API bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnor
  *           + s (q_t Hbar) sum_{U_i} alpha_tj
  *     D_t = sum_{S_i} sum_n e^{s q.k} + sum_{U_i} block * alpha_tj;   o_t = N_t / D_t
  *     (every exponent is shifted by a running row maximum, which cancels).
+ *   mode BSA_MODE_PISA_BLOCK ([PISA] §2, the per-block first-order term, of which the
+ *     Hbar form above is the global approximation):
+ *     N_t = sum_{S_i} sum_n e^{s q.k} v + sum_{U_i} alpha_tj (vsum_j + s q_t H_j)
+ *     D_t as for BSA_MODE_PISA. Because kbar_j is the mean key of block j, s q_t.kbar_j
+ *     is the mean of the row's exact scores over the block, and
+ *     alpha_tj (vsum_j + s q_t H_j) = sum_n alpha_tj (1 + s q_t.(k_{j,n} - kbar_j)) v_{j,n}:
+ *     every unselected block is computed as a tile whose weights are the first-order
+ *     expansion of e^{s q.k} about its centroid. No statistics are read (kbar, vsum,
+ *     Hbar may be NULL); every block of every query block is a tile, so the tensor
+ *     work is that of dense attention: an accuracy reference, not a fast path.
  *   Q, K, V      bf16 [Bt, H, L, d];   O bf16 [Bt, H, L, d] (written);
  *   row_ptr/col_idx  block lists, each row strictly ascending in [0, M);
  *     csr_per_head 0: one list of M rows (row_ptr int32[M+1]) shared by every head;
@@ -202,7 +213,7 @@ BSA_API bsa_status bsa_forward(const void* Q, const void* K, const void* V, int3
  *     so serialise them.
  *   - Returns BSA_ERR_SCRATCH_LIMIT when the shape needs more scratch than the array
  *     holds: PISA needs 256 + 2*BH*Mp*d*2 + BH*d*d*2 bytes (Mp = M rounded up to 128,
- *     each term rounded up to 256), keep-or-drop 256 bytes. Other errors as bsa_forward. */
+ *     each term rounded up to 256), the other modes 256 bytes. Other errors as bsa_forward. */
 BSA_API bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void* V, int32_t Bt,
                                        int32_t H, int32_t L, int32_t d, int32_t block,
                                        const int32_t* row_ptr, const int32_t* col_idx,

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libbsattn.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_BAD_CSR, ERR_TIMEOUT, ERR_WORKSPACE, \
     ERR_CAPACITY, ERR_SCRATCH_LIMIT = range(9)
 NOALLOC_SCRATCH_BYTES = 16 << 20
-MODE_KEEP_OR_DROP, MODE_PISA = 0, 1
+MODE_KEEP_OR_DROP, MODE_PISA, MODE_PISA_BLOCK = 0, 1, 2
 CALL_BUILD_MASK, CALL_PRECOMPUTE, CALL_ROUTE, CALL_FORWARD = 0, 1, 2, 3
 
 # Every symbol include/bsattn.h declares, in header order.

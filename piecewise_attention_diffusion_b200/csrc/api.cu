@@ -129,7 +129,8 @@ bsa_status bsa_forward(const void* Q, const void* K, const void* V, int32_t Bt, 
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return BSA_ERR_INVALID_ARG;
   if (csr_per_head != 0 && csr_per_head != 1) return BSA_ERR_INVALID_ARG;
-  if (mode != BSA_MODE_KEEP_OR_DROP && mode != BSA_MODE_PISA) return BSA_ERR_INVALID_ARG;
+  if (mode != BSA_MODE_KEEP_OR_DROP && mode != BSA_MODE_PISA && mode != BSA_MODE_PISA_BLOCK)
+    return BSA_ERR_INVALID_ARG;
   if (mode == BSA_MODE_PISA && (!kbar || !vsum || !Hbar)) return BSA_ERR_INVALID_ARG;
   if (!(scale >= 0.f)) return BSA_ERR_INVALID_ARG;
   const size_t need = bsa::forward_workspace(s);

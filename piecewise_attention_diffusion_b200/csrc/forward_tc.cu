@@ -77,6 +77,7 @@ struct Params {
   const int32_t* col_idx;
   int csr_per_head;
   int pisa;
+  int linear;  // per-block first order: every block a tile, unselected ones linearised
   float scale, scale_log2;
   __nv_bfloat16* O;
   float* lse;
@@ -157,7 +158,7 @@ struct StreamPos {
     qt = item % p.n_qt;
     lk = item_lists<QBPT>(p, bh, qt);
     lv = lk;
-    n_ex = count_exact<QBPT>(lk);
+    n_ex = p.linear ? p.M : count_exact<QBPT>(lk);
     n = n_ex + n_ch;
     t = 0;
   }
@@ -182,6 +183,37 @@ __device__ __forceinline__ float row_max(const uint32_t (&r)[128]) {
     m3 = max3(m3, __uint_as_float(r[e + 6]), __uint_as_float(r[e + 7]));
   }
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// Sum of the first N columns held in registers (packed adds in four chains).
+template <int N>
+__device__ __forceinline__ float row_sum(const uint32_t (&r)[128]) {
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int q = 0; q < N / 2; ++q)
+    acc[q & 3] = add2(acc[q & 3], make_float2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])));
+  const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+  return a.x + a.y;
+}
+
+// Linear weights c1 * s + c0 for the first N columns in r, written to TMEM as bf16 pairs
+// (column c holds elements 2c and 2c + 1) at p_addr.
+template <int N>
+__device__ __forceinline__ void row_lin(const uint32_t (&r)[128], float c1, float c0,
+                                        uint32_t p_addr) {
+  const float2 a = make_float2(c1, c1), b = make_float2(c0, c0);
+#pragma unroll
+  for (int h = 0; h < N / 64; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int e = h * 64 + 2 * q;
+      const float2 w = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a, b);
+      pk[q] = pack_bf16x2(w.x, w.y);
+    }
+    tmem_st32(p_addr + h * 32, pk);
+  }
 }
 
 // P for one row: 2^(s * scale_log2 - m_ref) for the first N columns in r, written to TMEM
@@ -229,7 +261,7 @@ struct Barriers {
   uint64_t done;
 };
 
-template <int D, int BKV>
+template <int D, int BKV, bool kLinear>
 __global__ void __launch_bounds__(kThreads, 1)
 k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
@@ -318,15 +350,17 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             s.advance(p, x, n_ch);
             return true;
           }
-          const bool r = s.n_ex > 0 ? load(kLoadK, s.lk.next(), s.bh) : load(kLoadKbar, 0, s.bh);
+          const bool r = s.n_ex > 0 ? load(kLoadK, p.linear ? 0 : s.lk.next(), s.bh)
+                                    : load(kLoadKbar, 0, s.bh);
           s.t = 1;
           return r;
         }
         const int u = s.t - 1;
-        if (!(u < s.n_ex ? load(kLoadV, s.lv.next(), s.bh) : load(kLoadVsum, u - s.n_ex, s.bh)))
+        if (!(u < s.n_ex ? load(kLoadV, p.linear ? u : s.lv.next(), s.bh)
+                         : load(kLoadVsum, u - s.n_ex, s.bh)))
           return false;
         if (s.t < s.n) {
-          const bool r = s.t < s.n_ex ? load(kLoadK, s.lk.next(), s.bh)
+          const bool r = s.t < s.n_ex ? load(kLoadK, p.linear ? s.t : s.lk.next(), s.bh)
                                       : load(kLoadKbar, s.t - s.n_ex, s.bh);
           ++s.t;
           return r;
@@ -503,7 +537,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int item = stream_item(k, x);
       const int bh = item / p.n_qt, qt = item % p.n_qt;
       Lists lists = item_lists<C::QBPT>(p, bh, qt);
-      const int n_ex = count_exact<C::QBPT>(lists);
+      const int n_ex = kLinear ? p.M : count_exact<C::QBPT>(lists);
       const int n = n_ex + n_ch;
       const int row_g = qt * kBQ + row;
       const int iq = qt * C::QBPT + row / BKV;   // this row's query block
@@ -512,6 +546,8 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       const int mb = has_blk ? __ldg(rp + iq) : 0;
       const int me = has_blk ? __ldg(rp + iq + 1) : 0;
       int mp = mb;
+      // per-block first order: the row's next selected block, fetched one match ahead
+      int nxt = kLinear && mp < me ? __ldg(p.col_idx + mp) : INT_MAX;
       float m_run = -INFINITY, l = 0.f, sa = 0.f;
 
       for (int t = 0; t < n; ++t) {
@@ -553,7 +589,15 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (!ok) break;
         tc_fence_after();
         bool skip = false;          // whole tile masked for this row
-        if (!chunk && C::QBPT == 2) {
+        bool lin = false;           // block t unselected for this row (per-block mode)
+        if (kLinear) {
+          if (nxt == t) {
+            ++mp;
+            nxt = mp < me ? __ldg(p.col_idx + mp) : INT_MAX;
+          } else {
+            lin = true;
+          }
+        } else if (!chunk && C::QBPT == 2) {
           const int j = lists.next();
           const bool member = mp < me && __ldg(p.col_idx + mp) == j;
           if (member) ++mp;
@@ -577,8 +621,12 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (int e = 0; e < 128; ++e)
               if ((excl[e >> 5] >> (e & 31)) & 1u) r[e] = __float_as_uint(-INFINITY);
           }
-          mx = cols == 128 ? row_max<128>(r) : row_max<64>(r);
+          if (kLinear && lin)  // the block's centroid score: the mean of its row scores
+            mx = (BKV == 128 ? row_sum<128>(r) : row_sum<64>(r)) * (1.0f / BKV);
+          else
+            mx = cols == 128 ? row_max<128>(r) : row_max<64>(r);
         }
+        const float mean = mx;
         mx *= p.scale_log2;
         const bool need = mx > m_run + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
@@ -611,6 +659,12 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           for (int e = 0; e < 32; ++e) z[e] = 0u;
           tmem_st32(s_base, z);
           if (cols == 128) tmem_st32(s_base + 32, z);
+        } else if (kLinear && lin) {
+          // first-order weights about the centroid: alpha (1 + s (score - mean)); the
+          // block adds B alpha to the denominator (its first-order part sums to zero)
+          const float alpha = ex2(mx - m_ref);
+          row_lin<BKV>(r, alpha * p.scale, alpha * (1.0f - p.scale * mean), s_base);
+          rs = (float)BKV * alpha;
         } else if (chunk) {
           rs = row_exp<128, false>(r, p.scale_log2, m_ref, s_base);
         } else {
@@ -769,7 +823,7 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool kLinear>
 cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, const void* vs16,
                 const void* hb16, cudaStream_t st) {
   using C = Cfg<D, BKV>;
@@ -799,24 +853,25 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.col_idx = a.col_idx;
   p.csr_per_head = a.csr_per_head;
   p.pisa = a.mode == BSA_MODE_PISA;
+  p.linear = a.mode == BSA_MODE_PISA_BLOCK;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.lse = a.lse;
   p.flag = flag;
   p.status = a.status;
-  cudaError_t e = cudaFuncSetAttribute(k_forward<D, BKV>,
+  cudaError_t e = cudaFuncSetAttribute(k_forward<D, BKV, kLinear>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc waits until the warpgroups that shrink have released enough registers:
   // the split must fit in what the launch allocates, or the kernel would never start
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, k_forward<D, BKV>);
+  e = cudaFuncGetAttributes(&fa, k_forward<D, BKV, kLinear>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs * kThreads < 128 * kRegsControl + 128 * kStreams * kRegsSoftmax)
     return cudaErrorInvalidConfiguration;
   const int grid = min(p.n_items, sm_count());
-  k_forward<D, BKV><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, p);
+  k_forward<D, BKV, kLinear><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, p);
   return cudaGetLastError();
 }
 
@@ -854,10 +909,18 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, const int32_t* flag, cudaStr
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (s.d == 64 && s.block == 64) return fwdtc::run<64, 64>(a, flag, kb16, vs16, hb16, st);
-  if (s.d == 64 && s.block == 128) return fwdtc::run<64, 128>(a, flag, kb16, vs16, hb16, st);
-  if (s.d == 128 && s.block == 64) return fwdtc::run<128, 64>(a, flag, kb16, vs16, hb16, st);
-  return fwdtc::run<128, 128>(a, flag, kb16, vs16, hb16, st);
+  // the per-block first-order mode is its own instantiation, so that the other modes'
+  // kernels carry none of its code (registers)
+  if (a.mode == BSA_MODE_PISA_BLOCK) {
+    if (s.d == 64 && s.block == 64) return fwdtc::run<64, 64, true>(a, flag, kb16, vs16, hb16, st);
+    if (s.d == 64 && s.block == 128) return fwdtc::run<64, 128, true>(a, flag, kb16, vs16, hb16, st);
+    if (s.d == 128 && s.block == 64) return fwdtc::run<128, 64, true>(a, flag, kb16, vs16, hb16, st);
+    return fwdtc::run<128, 128, true>(a, flag, kb16, vs16, hb16, st);
+  }
+  if (s.d == 64 && s.block == 64) return fwdtc::run<64, 64, false>(a, flag, kb16, vs16, hb16, st);
+  if (s.d == 64 && s.block == 128) return fwdtc::run<64, 128, false>(a, flag, kb16, vs16, hb16, st);
+  if (s.d == 128 && s.block == 64) return fwdtc::run<128, 64, false>(a, flag, kb16, vs16, hb16, st);
+  return fwdtc::run<128, 128, false>(a, flag, kb16, vs16, hb16, st);
 }
 
 }  // namespace bsa

@@ -69,10 +69,12 @@ extern "C" bsa_status bsa_forward_noalloc(const void* Q, const void* K, const vo
   if (!bsa::aligned16(Q) || !bsa::aligned16(K) || !bsa::aligned16(V) || !bsa::aligned16(O))
     return BSA_ERR_INVALID_ARG;
   if (csr_per_head != 0 && csr_per_head != 1) return BSA_ERR_INVALID_ARG;
-  if (mode != BSA_MODE_KEEP_OR_DROP && mode != BSA_MODE_PISA) return BSA_ERR_INVALID_ARG;
+  if (mode != BSA_MODE_KEEP_OR_DROP && mode != BSA_MODE_PISA && mode != BSA_MODE_PISA_BLOCK)
+    return BSA_ERR_INVALID_ARG;
   if (mode == BSA_MODE_PISA && (!kbar || !vsum || !Hbar)) return BSA_ERR_INVALID_ARG;
   if (!(scale >= 0.f)) return BSA_ERR_INVALID_ARG;
-  // keep-or-drop touches only the flag at the start of the scratch; PISA needs all of it
+  // keep-or-drop and the per-block mode touch only the flag at the start of the scratch;
+  // PISA needs all of it
   const size_t need = mode == BSA_MODE_PISA ? bsa::forward_workspace(s) : 256;
   if (need > (size_t)BSA_NOALLOC_SCRATCH_BYTES) return BSA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;

@@ -139,7 +139,7 @@ def _forward_check(w, q, k, v, rp, ci, per_head, mode, stats_np, qblocks=None, h
     scale = 1 / math.sqrt(w.head_dim)
     grp, gci = _csr_to_gpu(rp, ci)
     st = _status()
-    stats = _stats_to_gpu(*stats_np) if mode == b.MODE_PISA else None
+    stats = _stats_to_gpu(*stats_np[:3]) if mode == b.MODE_PISA else None
     O, lse = b.forward(q.to(DEV), k.to(DEV), v.to(DEV), w.block, grp, gci, per_head, mode,
                        stats=stats, want_lse=True, status=st)
     torch.cuda.synchronize()
@@ -152,9 +152,13 @@ def _forward_check(w, q, k, v, rp, ci, per_head, mode, stats_np, qblocks=None, h
         hrp, hci = orc.head_csr(rp, ci, h, M, per_head)
         blocks = list(range(M)) if qblocks is None else qblocks
         if mode == b.MODE_PISA:
-            kbar, vsum, Hbar = (x[h] for x in stats_np)
+            kbar, vsum, Hbar = (x[h] for x in stats_np[:3])
             want, wl = orc.pisa_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale, kbar,
                                      vsum, Hbar, qblocks=blocks)
+        elif mode == b.MODE_PISA_BLOCK:
+            kbar, vsum, Hbar, Hblk = (x[h] for x in stats_np)
+            want, wl = orc.pisa_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale, kbar,
+                                     vsum, Hbar, qblocks=blocks, Hblocks=Hblk)
         else:
             want, wl = orc.keep_or_drop_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale,
                                              qblocks=blocks)
@@ -283,6 +287,20 @@ def test_forward_growing_scores_exercise_the_rescale(mode):
         assert (np.abs(f64(lse[h]) - wl) <= ltol).all()
         print(f"[parity] grow mode={mode} head {h} max-abs {np.abs(got - want).max():.2e} "
               f"rel-L2 {rel_l2(got, want):.2e}")
+
+
+@pytest.mark.parametrize("L,block,d,kk", [(512, 64, 64, 2), (640, 128, 128, 2),
+                                          (1152, 64, 128, 5), (768, 128, 64, 6),
+                                          (128, 128, 128, 1)])
+def test_forward_pisa_per_block_first_order(L, block, d, kk):
+    """BSA_MODE_PISA_BLOCK against the oracle's per-block first-order PISA (each
+    unselected block's own H_j); lists from the oracle's routing."""
+    w = synth.Workload("perblock", 1, 3, L, d, block, "pisa", k_top=kk,
+                       generator="block_centres")
+    q, k, v = synth.make_qkv(w, seed=4)
+    kbar, vsum, H, Hbar, Mn = orc.precompute(f64(k), f64(v), block)
+    rp, ci, _ = orc.route(f64(q), kbar, Mn, block, kk, 1.0, 1 / math.sqrt(d))
+    _forward_check(w, q, k, v, rp, ci, 1, b.MODE_PISA_BLOCK, (kbar, vsum, Hbar, H))
 
 
 def test_forward_full_density_pisa_equals_keep_or_drop_equals_dense():
