@@ -44,17 +44,26 @@ def forward_flops(w, k_top: int, mode: str, row_lens=None) -> float:
     lens = [k_top] * M if row_lens is None else list(row_lens)
     total = 0.0
     for n in lens:
+        if mode == "pisa_block":  # every block is a tile (exact or linearised)
+            total += M * 4.0 * B * B * d
+            continue
         total += n * 4.0 * B * B * d
         if mode == "pisa":
             total += B * (4.0 * d * (M - n) + 2.0 * d * d)
     return w.batch * w.heads * total
 
 
+def needs_precompute(w) -> bool:
+    """The statistics feed the routing and PISA's Taylor tail; a fixed mask in the other
+    modes needs neither."""
+    return not w.mask or w.mode == "pisa"
+
+
 def launches_per_step(w) -> int:
     """Kernels one step launches: precompute 3 (statistics, reduce, norm; skipped for a
     fixed keep-or-drop mask), route 1 (not for a fixed mask), forward: list validation,
     the PISA statistics' bf16 conversion, the forward kernel."""
-    pre = 0 if (w.mask and w.mode != "pisa") else 3
+    pre = 3 if needs_precompute(w) else 0
     route = 0 if w.mask else 1
     fwd = 3 if w.mode == "pisa" else 2
     return pre + route + fwd
@@ -205,6 +214,13 @@ def load_traffic(w) -> float | None:
 
 
 # -------------------------------------------------------------- CPU oracle timing
+def _steps_done(w) -> str:
+    done = (["precomputed"] if (not w.mask or w.mode != "keep_or_drop") else []) \
+        + ([] if w.mask else ["routed"]) + ["attended"]
+    return ", ".join(done[:-1]) + (" and " if len(done) > 1 else "") + done[-1]
+
+
+
 def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
     """Time the fp64 oracle (as it stands) on `heads_sample` full heads and scale to
     the whole workload by the head count."""
@@ -221,7 +237,7 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
     t0 = time.perf_counter()
     for h in heads:
         qf, kf, vf = (x[h].to(torch.float64).numpy() for x in (q, k, v))
-        if fixed is not None and w.mode != "pisa":
+        if fixed is not None and w.mode == "keep_or_drop":
             orc.keep_or_drop_head(qf, kf, vf, fixed[0], fixed[1], w.block, scale)
             continue
         kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block)
@@ -231,15 +247,16 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
             rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale)
         if w.mode == "pisa":
             orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar)
+        elif w.mode == "pisa_block":
+            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar, Hblocks=H)
         else:
             orc.keep_or_drop_head(qf, kf, vf, rp, ci, w.block, scale)
     dt = time.perf_counter() - t0
     BH = w.batch * w.heads
     return {"seconds_sample": dt, "seconds_full_est": dt * BH / len(heads), "cores": threads,
-            "sample": f"{len(heads)} of {BH} heads, each fully "
-                      f"{'precomputed and ' if (w.mode == 'pisa' or not w.mask) else ''}"
-                      f"{'' if w.mask else 'routed and '}attended (all {w.n_blocks} query "
-                      f"blocks{', fixed mask' if w.mask else ''}); time scaled by heads"}
+            "sample": f"{len(heads)} of {BH} heads, each fully {_steps_done(w)} (all "
+                      f"{w.n_blocks} query blocks{', fixed mask' if w.mask else ''}); "
+                      f"time scaled by heads"}
 
 
 # --------------------------------------------------------------------- our arm
@@ -271,13 +288,13 @@ def run_ours(args, w, world, rank, local):
     O = torch.empty_like(qd)
     ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
     ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
-    mode = b.MODE_PISA if w.mode == "pisa" else b.MODE_KEEP_OR_DROP
+    mode = {"pisa": b.MODE_PISA, "pisa_block": b.MODE_PISA_BLOCK}.get(w.mode, b.MODE_KEEP_OR_DROP)
     stream = torch.cuda.current_stream(dev)
 
     def step(qx, kx, vx, ev=None):
         if ev:
             ev[0].record(stream)
-        if not (w.mask and mode != b.MODE_PISA):
+        if needs_precompute(w):
             b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
                              stats["Mnorm"], None, ws_p, st)
         if ev:
@@ -322,7 +339,7 @@ def run_ours(args, w, world, rank, local):
         raise RuntimeError(f"device status {b.status_string(st.item())}")
 
     F_fwd = forward_flops(w, k_top, w.mode, row_lens)
-    F_step = F_fwd + (0.0 if (w.mask and w.mode != "pisa") else precompute_flops(w)) \
+    F_step = F_fwd + (precompute_flops(w) if needs_precompute(w) else 0.0) \
         + (0.0 if w.mask else route_flops(w))
     value = world * F_step / (ms_step * 1e-3) / 1e12
     pk = peaks()
@@ -406,7 +423,7 @@ def run_reference(args, w, world, rank):
         rp, _ = orc.dense_to_csr(orc.mask_dense(**w.mask))
         row_lens = np.diff(rp).tolist()
     F_step = forward_flops(w, k_top, w.mode, row_lens) \
-        + (0.0 if (w.mask and w.mode != "pisa") else precompute_flops(w)) \
+        + (precompute_flops(w) if needs_precompute(w) else 0.0) \
         + (0.0 if w.mask else route_flops(w))
     for _ in range(args.warmup):
         oracle_sample(w, k_top, 1, args.seed)

@@ -13,6 +13,7 @@ Workloads (sizes named after what they are):
   * multimodal_dit     batch 8, 16 heads, L=1152 (77 text tokens padded to 128 +
                        32x32 image patches), d=64, block 64
   * multimodal_pisa    the same shape and fixed mask as the exact set of PISA
+  * image_pisa_block, video_pisa_block   the per-block first-order form of PISA
   * image_pisa         batch 1, 24 heads, L=4096 (64x64 latent), d=128, block 128
   * video_pisa         batch 1, 40 heads, L=16384 (16 frames x 32x32), d=128, block 128
   * sweep_L{L}         batch 1, 24 heads, L in {4096..32768}, d=128, block 128
@@ -34,7 +35,7 @@ class Workload:
     seq_len: int
     head_dim: int
     block: int
-    mode: str                    # "pisa" or "keep_or_drop"
+    mode: str                    # "pisa", "pisa_block" or "keep_or_drop"
     density: float | None = None  # fraction of KV blocks computed exactly (routing)
     k_top: int | None = None      # explicit top-k (overrides density)
     generator: str = "iid"        # iid | block_centres | field2d_hot | field3d
@@ -71,6 +72,11 @@ def workloads() -> dict:
                                generator="field2d_hot", grid=(64, 64))
     w["video_pisa"] = Workload("video_pisa", 1, 40, 16384, 128, 128, "pisa", density=0.125,
                                generator="field3d", grid=(16, 32, 32))
+    # the per-block first-order form of PISA (every block a tile: dense tensor work)
+    w["image_pisa_block"] = dataclasses.replace(w["image_pisa"], name="image_pisa_block",
+                                                mode="pisa_block")
+    w["video_pisa_block"] = dataclasses.replace(w["video_pisa"], name="video_pisa_block",
+                                                mode="pisa_block")
     for L in (4096, 8192, 16384, 32768):
         for dens in (1.0, 0.25, 0.125):
             for mode in ("keep_or_drop", "pisa"):
