@@ -12,11 +12,12 @@
 // and the epilogue thread that owns row a of C applies the centring in fp32:
 //     H_j[a][c] = C_j[a][c] - (ksum_j[a] / B) * vsum_j[c].
 // Two passes over K and V, because M_j needs H-bar, i.e. every block of the head:
-//   stats pass  writes kbar, vsum and, per group of kGroup blocks, the partial sum of
-//               H_j (the group's rows kept in registers; written once per group);
+//   stats pass  writes kbar, vsum and, per head segment of its range, the partial sum
+//               of H_j (rows kept in registers; written once per segment);
 //   (a reduce kernel then forms H-bar from the partials in a fixed order);
 //   norm pass   recomputes H_j and reduces ||H_j - H-bar||_F over the 128 rows.
-// Each pass is one persistent kernel over contiguous ranges of blocks (so a CTA meets
+// Each pass is one persistent kernel; the flattened (head, block) range is dealt in
+// contiguous pieces of equal length, one per CTA (so every SM works, and a CTA meets
 // few heads and reloads H-bar rarely): warp 0 issues TMA into a 3-stage ring of (K_j,
 // V_j) pairs, warp 1 issues the MMAs into two TMEM buffers, warps 2-5 run the epilogue.
 // Every mbarrier wait is bounded; a timeout aborts the CTA and reports BSA_ERR_TIMEOUT.
@@ -34,7 +35,7 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int kThreads = 192;
 constexpr int kStages = 3;
-constexpr int kGroup = 8;  // blocks per partial sum of H_j (stats pass)
+constexpr int kMaxGrid = 256;  // CTAs per pass at most (bounds the partial-sum workspace)
 constexpr uint32_t kTmemCols = 512;
 // TMEM buffer b: C at 256 b, ksum at 256 b + 128, vsum at 256 b + 144 (16 columns each)
 
@@ -48,53 +49,39 @@ struct Cfg {
 
 struct Params {
   int L, M, BH;
-  int n_units, per_cta;   // units: groups of kGroup blocks (stats) or blocks (norm)
-  bool stats;             // unit = group of kGroup blocks (stats pass) or one block
+  int n_units, per_cta;   // units = blocks (b*H + h) * M + j; CTA c takes [c per_cta, ..)
+  bool stats;
   float* kbar;
   float* vsum;
-  float* partial;         // stats: [BH, ceil(M / kGroup), D, D]
+  float* partial;         // stats: slot c + bh per (CTA c, head bh) segment, [., D, D]
   const float* Hbar;      // norm
   float* Mnorm;           // norm
   float* Hblk;            // norm, nullable
   int32_t* status;
 };
 
-// The blocks this CTA processes, in order: unit range [u0, u1) of the pass.
+// The blocks this CTA processes, in order: the contiguous range [u0, u1) of the pass.
+// A head segment is the run of the range's blocks that belong to one head.
 struct BlockIter {
-  int u, u1, j, j1, bh;
-  bool stats;
-  int M, n_grp;
+  int u, u1, j, bh, M;
   __device__ __forceinline__ void init(const Params& p) {
-    stats = p.stats;
     M = p.M;
-    n_grp = ceil_div(p.M, kGroup);
     u = blockIdx.x * p.per_cta;
     u1 = min(p.n_units, u + p.per_cta);
-    j = j1 = 0;
-    bh = 0;
-    load_unit();
-  }
-  __device__ __forceinline__ void load_unit() {
-    if (u >= u1) return;
-    if (stats) {
-      bh = u / n_grp;
-      const int g = u % n_grp;
-      j = g * kGroup;
-      j1 = min(M, j + kGroup);
-    } else {
-      bh = u / M;
-      j = u % M;
-      j1 = j + 1;
-    }
+    bh = u / M;
+    j = u % M;
   }
   __device__ __forceinline__ bool valid() const { return u < u1; }
-  // advance to the next block; returns true when a unit (group) just ended
+  // advance to the next block; returns true when a head segment just ended
   __device__ __forceinline__ bool next() {
-    ++j;
-    if (j < j1) return false;
     ++u;
-    load_unit();
-    return true;
+    ++j;
+    if (j == M) {
+      j = 0;
+      ++bh;
+      return true;
+    }
+    return u >= u1;
   }
 };
 
@@ -221,8 +208,7 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int quad = warp % 4;
     const int a = quad * 32 + lane;              // row of C = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const int n_grp = ceil_div(p.M, kGroup);
-    // stats: partial sum of H_j row a over the group; norm: H-bar row a of the head
+    // stats: partial sum of H_j row a over the head segment; norm: H-bar row a of the head
     float acc[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) acc[c] = 0.f;
@@ -315,9 +301,11 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       ++n;
       const bool unit_end = it.next();
       if (kStats && unit_end) {
-        // group finished: write its partial sum (row a) and start a new one
-        const int g = j / kGroup;
-        float4* dst = reinterpret_cast<float4*>(p.partial + (((size_t)bh * n_grp + g) * D + a) * D);
+        // head segment finished: write its partial sum (row a) into slot blockIdx.x + bh
+        // (distinct per (CTA, head): the next CTA's first head is at least this one's
+        // last) and start a new one
+        float4* dst = reinterpret_cast<float4*>(
+            p.partial + (((size_t)blockIdx.x + bh) * D + a) * D);
 #pragma unroll
         for (int c = 0; c < D / 4; ++c) {
           dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
@@ -336,15 +324,19 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   }
 }
 
-// H-bar = (1 / M) * sum of the partial sums of one head, in a fixed order.
-__global__ void k_reduce(const float* __restrict__ partial, int n_grp, int M,
+// H-bar = (1 / M) * sum of the head's segment partial sums, in CTA order (fixed for a
+// given grid: deterministic). CTA c covers blocks [c per, (c + 1) per) of the flattened
+// (head, block) range, so head bh's segments come from CTAs bh M / per ..
+// ((bh + 1) M - 1) / per, and CTA c wrote its segment of head bh into slot c + bh.
+__global__ void k_reduce(const float* __restrict__ partial, int per, int grid, int M,
                          float* __restrict__ Hbar) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int bh = blockIdx.y;
   if (e >= D * D) return;
-  const float* q = partial + (size_t)bh * n_grp * D * D + e;
+  const int c0 = (int)((int64_t)bh * M / per);
+  const int c1 = min(grid - 1, (int)(((int64_t)bh * M + M - 1) / per));
   float s = 0.f;
-  for (int g = 0; g < n_grp; ++g) s += q[(size_t)g * D * D];
+  for (int c = c0; c <= c1; ++c) s += partial[((size_t)c + bh) * D * D + e];
   Hbar[(size_t)bh * D * D + e] = s / (float)M;
 }
 
@@ -402,7 +394,7 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   e = cudaFuncSetAttribute(k_precompute<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Cf::SMEM);
   if (e != cudaSuccess) return e;
-  const int M = s.M(), n_grp = ceil_div(M, kGroup), sms = sm_count();
+  const int M = s.M(), sms = std::min(sm_count(), kMaxGrid);
   Params p;
   p.L = s.L;
   p.M = M;
@@ -414,26 +406,28 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   p.Mnorm = Mnorm;
   p.Hblk = Hblk;
   p.status = status;
-  // stats pass over groups of kGroup blocks
-  p.stats = true;
-  p.n_units = s.BH() * n_grp;
-  p.per_cta = ceil_div(p.n_units, sms);
-  k_precompute<B, true><<<ceil_div(p.n_units, p.per_cta), kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_reduce<<<dim3(ceil_div(D * D, 256), s.BH()), 256, 0, st>>>(p.partial, n_grp, M, Hbar);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // norm pass over single blocks
-  p.stats = false;
+  // both passes deal the flattened (head, block) range in contiguous pieces, one per CTA
   p.n_units = s.BH() * M;
   p.per_cta = ceil_div(p.n_units, sms);
-  k_precompute<B, false><<<ceil_div(p.n_units, p.per_cta), kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
+  const int grid = ceil_div(p.n_units, p.per_cta);
+  p.stats = true;
+  k_precompute<B, true><<<grid, kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_reduce<<<dim3(ceil_div(D * D, 256), s.BH()), 256, 0, st>>>(p.partial, p.per_cta, grid, M,
+                                                                 Hbar);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  p.stats = false;
+  k_precompute<B, false><<<grid, kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
   return cudaGetLastError();
 }
 
 }  // namespace pretc
 
 size_t precompute_tc_workspace(const Shape& s) {
-  return (size_t)s.BH() * ceil_div(s.M(), pretc::kGroup) * pretc::D * pretc::D * sizeof(float);
+  // one partial sum per (CTA, head) segment: at most grid + BH - 1 slots, grid <= kMaxGrid
+  // and <= the number of blocks
+  const size_t grid = std::min<size_t>(pretc::kMaxGrid, (size_t)s.BH() * s.M());
+  return (grid + s.BH()) * pretc::D * pretc::D * sizeof(float);
 }
 
 cudaError_t launch_precompute_tc(const Shape& s, const void* K, const void* V, float* kbar,
