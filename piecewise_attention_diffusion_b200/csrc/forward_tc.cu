@@ -53,6 +53,7 @@ using namespace sm100;
 constexpr int kBQ = 128;       // query rows per tile
 constexpr int kChunk = 128;    // centroids per sweep tile
 constexpr int kStreams = 2;                   // query tiles in flight per CTA
+static_assert(kStreams == 2, "the issuer's Q descriptor table holds two streams");
 constexpr int kThreads = 128 * (kStreams + 1);  // softmax warpgroups, then a control warpgroup
 constexpr int kProducerWarp = 4 * kStreams;      // first warp of the control warpgroup
 constexpr int kMmaWarp = kProducerWarp + 1;      // (its two other warps only idle)
@@ -394,29 +395,38 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      uint32_t ring = 0;
+      // ring position as (slot, phase), advanced without division; `last` is the slot
+      // of the most recent wait_slot
+      uint32_t slot = 0, phase = 0, last = 0;
       bool ok = true;
       constexpr uint32_t idesc_s_ex = idesc_bf16_f32(kBQ, BKV, false, false);
       constexpr uint32_t idesc_s_ch = idesc_bf16_f32(kBQ, kChunk, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, D, false, true);
       auto wait_slot = [&](uint32_t& addr) -> bool {
-        const int slot = ring % C::NSLOT;
-        if (!mbar_wait(&bars.kv_full[slot], (ring / C::NSLOT) & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars.kv_full[slot], phase, abort_flag)) return false;
         tc_fence_after();
         addr = smem_u32(sSlot + slot * C::SLOT);
-        ++ring;
+        last = slot;
+        if (++slot == (uint32_t)C::NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
         return true;
       };
-      auto release_slot = [&]() { mma_commit(&bars.kv_empty[(ring - 1) % C::NSLOT]); };
+      auto release_slot = [&]() { mma_commit(&bars.kv_empty[last]); };
+      // A descriptor's start-address field is the address in 16-byte units (the shared
+      // window is below 256 KB, so the 14-bit field never carries): the descriptor of
+      // a K-step is the tile's descriptor plus its byte offset / 16.
+      const uint64_t qdesc[kStreams] = {smem_desc_sw128(smem_u32(smem), 16, 1024),
+                                        smem_desc_sw128(smem_u32(smem + C::QBYTES), 16, 1024)};
       // S = Q K^T (K-major operands) into the stream's S buffer
       auto issue_s = [&](int x, uint32_t k_addr, int rows, uint32_t idesc) {
-        const uint32_t q_addr = smem_u32(smem + x * C::QBYTES);
+        const uint64_t a0 = x ? qdesc[1] : qdesc[0];
+        const uint64_t b0 = smem_desc_sw128(k_addr, 16, 1024);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint64_t adesc =
-              smem_desc_sw128(q_addr + (k / 4) * (kBQ * 128) + (k % 4) * 32, 16, 1024);
-          const uint64_t bdesc =
-              smem_desc_sw128(k_addr + (k / 4) * (rows * 128) + (k % 4) * 32, 16, 1024);
+          const uint64_t adesc = a0 + (uint64_t)(((k / 4) * (kBQ * 128) + (k % 4) * 32) >> 4);
+          const uint64_t bdesc = b0 + (uint64_t)(((k / 4) * (rows * 128) + (k % 4) * 32) >> 4);
           mma_ss(tmem + C::S_COL(x), adesc, bdesc, idesc, k > 0 ? 1u : 0u);
         }
       };
@@ -443,43 +453,44 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           s.t = 1;
           return true;
         }
-        // PV(u) with P (bf16, TMEM) of tile u
+        // PV(u) with P (bf16, TMEM) of tile u, then S(t): both operands' waits first, so
+        // that the step's MMAs go out back to back
         const int u = s.t - 1;
         if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag)) return false;
         tc_fence_after();
-        uint32_t v_addr;
+        uint32_t v_addr, k_addr = 0;
         if (!wait_slot(v_addr)) return false;
+        const uint32_t v_slot = last;
+        const bool more = s.t < s.n;
+        if (more && !wait_slot(k_addr)) return false;
         {
           const int kdim = u >= s.n_ex ? kChunk : BKV;
-          for (int k = 0; k < kdim / 16; ++k) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + k * 2048, kdim * 128, 1024);
-            mma_ts(tmem + C::O_COL(x), tmem + C::S_COL(x) + k * 8, bdesc, idesc_o,
-                   (u > 0 || k > 0) ? 1u : 0u);
-          }
+          const uint64_t b0 = smem_desc_sw128(v_addr, kdim * 128, 1024);
+          for (int k = 0; k < kdim / 16; ++k)
+            mma_ts(tmem + C::O_COL(x), tmem + C::S_COL(x) + k * 8, b0 + (uint64_t)(k * 128),
+                   idesc_o, (u > 0 || k > 0) ? 1u : 0u);
         }
-        release_slot();
-        if (s.t < s.n) {
-          uint32_t k_addr;
-          if (!wait_slot(k_addr)) return false;
+        if (more) {
           const bool chunk = s.t >= s.n_ex;
           issue_s(x, k_addr, chunk ? kChunk : BKV, chunk ? idesc_s_ch : idesc_s_ex);
+          mma_commit(&bars.kv_empty[v_slot]);
           release_slot();
           mma_commit(&bars.s_full[x]);
           ++s.t;
           return true;
         }
+        mma_commit(&bars.kv_empty[v_slot]);
         if (p.pisa) {
           // first-order term T = Q Hbar into this stream's (now free) S buffer
           uint32_t h_addr;
           if (!wait_slot(h_addr)) return false;
-          const uint32_t q_addr = smem_u32(smem + x * C::QBYTES);
+          const uint64_t a0 = x ? qdesc[1] : qdesc[0];
+          const uint64_t b0 = smem_desc_sw128(h_addr, D * 128, 1024);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t adesc =
-                smem_desc_sw128(q_addr + (k / 4) * (kBQ * 128) + (k % 4) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(h_addr + k * 2048, D * 128, 1024);
-            mma_ss(tmem + C::S_COL(x), adesc, bdesc, idesc_o, k > 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < D / 16; ++k)
+            mma_ss(tmem + C::S_COL(x),
+                   a0 + (uint64_t)(((k / 4) * (kBQ * 128) + (k % 4) * 32) >> 4),
+                   b0 + (uint64_t)(k * 128), idesc_o, k > 0 ? 1u : 0u);
           release_slot();
         }
         mma_commit(&bars.o_final[x]);
