@@ -11,9 +11,9 @@
 // One CTA per (head, 8 query blocks), one warp per query block:
 //   1. pooled query: the warp streams its block of Q with 16-byte loads (the only HBM
 //      stream of the call) and reduces the columns;
-//   2. scores: the head's centroids are staged through shared memory in chunks of 64
-//      rows (rows padded to D+1 floats so that 32 lanes reading 32 centroids hit 32
-//      banks) and each lane dots its centroids with the pooled query;
+//   2. scores: thread t takes centroid j = t (looping when M > 256), reads its row once
+//      per CTA (16-byte loads from L2) and dots it with the CTA's 8 pooled queries, which
+//      every thread reads from the same shared-memory words (broadcast);
 //   3. softmax over the M blocks plus the normalised covariance term;
 //   4. exact top-k: the k-th largest score is found by a radix select on the float bit
 //      patterns (scores are >= 0, so the bit patterns order like the values), ties at
@@ -27,7 +27,6 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunkC = 64;  // centroids per staged chunk
 
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
@@ -41,9 +40,8 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   const int i = blockIdx.x * kWarps + warp;  // this warp's query block
   const bool active = i < M;
 
-  extern __shared__ float smem[];
-  float* s_kb = smem;                           // kChunkC x (D + 1)
-  float* s_q = s_kb + kChunkC * (D + 1);        // kWarps x D
+  extern __shared__ __align__(16) float smem[];
+  float* s_q = smem;                            // kWarps x D (16-byte aligned rows)
   float* s_cov = s_q + kWarps * D;              // M
   float* s_sc = s_cov + M;                      // kWarps x M
   float* s_red = s_sc + kWarps * M;             // kWarps
@@ -89,50 +87,40 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   }
   __syncwarp();
 
-  // 2. block scores a_j = scale * qbar . kbar_j, centroids staged 64 at a time
+  // 2. block scores a_j = scale * qbar_w . kbar_j for the CTA's query blocks
   const float* kb = kbar + (size_t)bh * M * D;
   float* sc = s_sc + warp * M;
-  // 16-byte loads when the caller's kbar allows them (each head's slice then does too,
-  // since M * D * 4 is a multiple of 16); unrolled so that a thread's loads are in flight
-  // together rather than one L2 round trip after another
-  const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
-  for (int c0 = 0; c0 < M; c0 += kChunkC) {
-    const int nc = min(kChunkC, M - c0);
-    __syncthreads();
-    if (vec) {
-      const float4* src = reinterpret_cast<const float4*>(kb + (size_t)c0 * D);
-#pragma unroll 8
-      for (int e4 = threadIdx.x; e4 < nc * D / 4; e4 += kThreads) {
-        const float4 v = __ldg(src + e4);
-        float* dst = s_kb + (e4 * 4 / D) * (D + 1) + (e4 * 4 % D);
-        dst[0] = v.x;
-        dst[1] = v.y;
-        dst[2] = v.z;
-        dst[3] = v.w;
-      }
-    } else {
-#pragma unroll 8
-      for (int e = threadIdx.x; e < nc * D; e += kThreads) {
-        const int r = e / D, c = e % D;
-        s_kb[r * (D + 1) + c] = __ldg(kb + (size_t)(c0 + r) * D + c);
-      }
-    }
-    __syncthreads();
-    if (active) {
-      for (int jj = lane; jj < nc; jj += 32) {
-        const float* kr = s_kb + jj * (D + 1);
-        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-#pragma unroll 8
-        for (int c = 0; c < D; c += 4) {
-          d0 = fmaf(qbar[c], kr[c], d0);
-          d1 = fmaf(qbar[c + 1], kr[c + 1], d1);
-          d2 = fmaf(qbar[c + 2], kr[c + 2], d2);
-          d3 = fmaf(qbar[c + 3], kr[c + 3], d3);
-        }
-        sc[c0 + jj] = scale * ((d0 + d1) + (d2 + d3));
-      }
-    }
+  if (!active) {
+#pragma unroll 1
+    for (int c = lane; c < D; c += 32) qbar[c] = 0.f;  // keep the dots below finite
   }
+  __syncthreads();
+  // 16-byte loads when the caller's kbar allows them (each head's slice then does too,
+  // since M * D * 4 is a multiple of 16)
+  const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
+  for (int j = threadIdx.x; j < M; j += kThreads) {
+    float acc[kWarps];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) acc[w] = 0.f;
+    const float* kr = kb + (size_t)j * D;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      float4 kv;
+      if (vec) {
+        kv = __ldg(reinterpret_cast<const float4*>(kr + c));
+      } else {
+        kv = make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2), __ldg(kr + c + 3));
+      }
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float4 qv = *reinterpret_cast<const float4*>(s_q + w * D + c);
+        acc[w] = fmaf(qv.w, kv.w, fmaf(qv.z, kv.z, fmaf(qv.y, kv.y, fmaf(qv.x, kv.x, acc[w]))));
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s_sc[w * M + j] = scale * acc[w];
+  }
+  __syncthreads();
   __syncwarp();
   if (!active) return;
 
@@ -194,9 +182,7 @@ cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* M
                 int k_top, float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
                 float* scores, cudaStream_t st) {
   const int M = s.M();
-  const size_t sm =
-      ((size_t)kChunkC * (D + 1) + (size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) *
-      sizeof(float);
+  const size_t sm = ((size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(k_route<B, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
