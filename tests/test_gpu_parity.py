@@ -371,15 +371,27 @@ def test_forward_malformed_lists_set_status_and_leave_output():
 @pytest.mark.parametrize("name,heads,qblocks", [
     ("image_pisa", [0, 13], None),
     ("video_pisa", [0, 39], [0, 1, 63, 127]),
+    ("sweep_L32768_d125_pisa", [0, 23], [0, 100, 255]),
 ])
 def test_pipeline_full_size_sampled(name, heads, qblocks):
-    """precompute -> route -> forward on the GPU over the full workload, in the launch
+    _pipeline_sampled(synth.workloads()[name], heads, qblocks)
+
+
+def test_pipeline_maximum_blocks():
+    """The largest block count the library accepts (M = 2048: L = 262144 at block 128):
+    sixteen centroid chunks in the sweep, a 2048-wide radix select in routing."""
+    w = synth.Workload("max_blocks", 1, 1, 2048 * 128, 128, 128, "pisa", k_top=64,
+                       generator="field3d", grid=(256, 32, 32))
+    _pipeline_sampled(w, [0], [0, 1000, 2047])
+
+
+def _pipeline_sampled(w, heads, qblocks):
+    """precompute -> route -> forward on the GPU over the whole workload, in the launch
     configuration the benchmark uses; the oracle checks the sampled heads.
 
     The forward for the sampled heads is run on the oracle's own block lists (spliced
     into the GPU-routed lists), so the output comparison does not depend on near-tie
     routing decisions; the routing itself is compared separately with the tie rule."""
-    w = synth.workloads()[name]
     q, k, v = synth.make_qkv(w)
     kk, M, BH = w.top_k(), w.n_blocks, w.batch * w.heads
     scale = 1 / math.sqrt(w.head_dim)
@@ -412,6 +424,6 @@ def test_pipeline_full_size_sampled(name, heads, qblocks):
     for h in heads:
         blocks = list(range(M)) if qblocks is None else qblocks
         rows = np.concatenate([np.arange(i * w.block, (i + 1) * w.block) for i in blocks])
-        mx, rl = assert_close_out(Og[h, rows], ref[h][0], f"{name} head {h}")
-        print(f"[parity] {name} head {h} max-abs {mx:.2e} rel-L2 {rl:.2e}")
+        mx, rl = assert_close_out(Og[h, rows], ref[h][0], f"{w.name} head {h}")
+        print(f"[parity] {w.name} head {h} max-abs {mx:.2e} rel-L2 {rl:.2e}")
     assert torch.isfinite(O.float()).all()
