@@ -177,11 +177,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's x (the slowest rank's time), on every rank. The tensor
+    lives where the process group's backend needs it (NCCL: this rank's GPU)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(flops_per_rank: float, ms_slowest: float, world: int) -> float:
+    """Whole-job TFLOP/s of `world` replicas that each ran `flops_per_rank` per step, timed
+    by the slowest rank (weak scaling: every rank does the full workload)."""
+    return world * flops_per_rank / (ms_slowest * 1e-3) / 1e12
 
 
 def peaks() -> dict:
@@ -341,7 +350,7 @@ def run_ours(args, w, world, rank, local):
     F_fwd = forward_flops(w, k_top, w.mode, row_lens)
     F_step = F_fwd + (precompute_flops(w) if needs_precompute(w) else 0.0) \
         + (0.0 if w.mask else route_flops(w))
-    value = world * F_step / (ms_step * 1e-3) / 1e12
+    value = replica_value(F_step, ms_step, world)
     pk = peaks()
     achieved = F_fwd / (fwd_ms * 1e-3) / 1e12
 
@@ -371,7 +380,7 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world)
-        e2e = {"value": round(world * F_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e2e = {"value": round(replica_value(F_step, e2e_ms, world), 3), "unit": "TFLOP/s",
                "ms_per_step": round(e2e_ms, 4),
                "h2d_bytes_per_step": int(3 * q.numel() * 2),
                "d2h_bytes_per_step": int(O.numel() * 2)}
