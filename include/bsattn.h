@@ -222,6 +222,16 @@ BSA_API bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void*
                                        float scale, void* O, float* lse, int32_t* status,
                                        void* stream);
 
+/* bsa_selftest_wait_timeout — the failure path of every kernel, exercised without a fault.
+ * (No counterpart in the pages.) Every wait of the library's kernels is bounded: a wait
+ * that runs out sets a CTA-wide abort flag, the kernel drains and returns, and
+ * BSA_ERR_TIMEOUT is written to *status, leaving the context usable. This call launches
+ * one CTA whose thread waits, with that same bounded wait and a limit of timeout_ns, on
+ * an mbarrier that nothing ever completes; the wait runs out and the kernel reports.
+ *   timeout_ns  1 .. 10^10 (10 s); status: device int32, written with BSA_ERR_TIMEOUT.
+ * Returns BSA_ERR_INVALID_ARG for a null status or a limit out of range. */
+BSA_API bsa_status bsa_selftest_wait_timeout(int64_t timeout_ns, int32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

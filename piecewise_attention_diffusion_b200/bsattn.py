@@ -29,7 +29,7 @@ CALL_BUILD_MASK, CALL_PRECOMPUTE, CALL_ROUTE, CALL_FORWARD = 0, 1, 2, 3
 # Every symbol include/bsattn.h declares, in header order.
 EXPORTS = ("bsa_version", "bsa_status_string", "bsa_mask_blocks", "bsa_workspace_bytes",
            "bsa_build_mask", "bsa_precompute", "bsa_route", "bsa_forward",
-           "bsa_forward_noalloc")
+           "bsa_forward_noalloc", "bsa_selftest_wait_timeout")
 
 
 class BsaError(RuntimeError):
@@ -61,6 +61,7 @@ _SIGS = {
                            _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
                                    _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp]),
+    "bsa_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
 }
 
 
@@ -228,6 +229,14 @@ def bsa_forward_noalloc(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kb
                                      int(csr_per_head), int(mode), _ptr(kbar), _ptr(vsum),
                                      _ptr(Hbar), float(scale), _ptr(O), _ptr(lse),
                                      _ptr(status), _stream(stream)), "bsa_forward_noalloc")
+
+
+def bsa_selftest_wait_timeout(timeout_ns, status, stream=None):
+    """Launch the bounded-wait self-test: the kernel's wait runs out after timeout_ns and
+    BSA_ERR_TIMEOUT is written to `status` (device int32)."""
+    _need(status, torch.int32, "status")
+    _check(lib().bsa_selftest_wait_timeout(int(timeout_ns), _ptr(status), _stream(stream)),
+           "bsa_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------ allocating helpers
