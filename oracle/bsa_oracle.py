@@ -31,7 +31,15 @@ Readings taken where the pages are silent:
   * routing score_ij = softmax_j(s qbar_i . kbar_j) + lambda * M_j / sum_j' M_j',
     qbar_i = mean of the block's queries; top-k by descending score, ties to the
     smaller j; lists emitted in ascending j;
-  * a keep-or-drop row with an empty list outputs zeros (lse = -inf).
+  * a keep-or-drop row with an empty list outputs zeros (lse = -inf);
+  * token-level padding ([BSA] §4.1 pads the text segment to a multiple of the block
+    size; §7.3 gives a timestep token its own block): ``key_valid[j]`` is the number of
+    leading real tokens of block j (the rest are padding). Padded keys get no weight;
+    centroids, value sums, H_j and pooled queries are taken over the real tokens; an
+    unselected block's Taylor-tail weight is its number of real tokens; a padded block
+    is always in S_i (routing places it there first), since a partial block's centroid
+    is a poor expansion point and the pages keep such blocks fully connected anyway.
+    Padded query rows are computed like any other row.
 
 Parity pins live in tests/test_oracle.py. The overall approximation error of PISA
 against dense attention is parity unpinned by the pages (they print no error
@@ -90,6 +98,18 @@ def _row(row_ptr, col_idx, i):
     return [int(c) for c in col_idx[row_ptr[i]:row_ptr[i + 1]]]
 
 
+def _valid(key_valid, M, block):
+    """Real tokens per block (all of them when there is no padding)."""
+    return [block] * M if key_valid is None else [int(x) for x in key_valid]
+
+
+def _keys(blocks, block, valid):
+    """Token positions of the real keys of the given blocks, in order."""
+    if not blocks:
+        return np.zeros(0, dtype=np.int64)
+    return np.concatenate([np.arange(j * block, j * block + valid[j]) for j in blocks])
+
+
 # ----------------------------------------------------------------------------------
 # Dense softmax attention (reference for the approximation error)
 # ----------------------------------------------------------------------------------
@@ -105,8 +125,9 @@ def dense_head(q, k, v, scale):
 # ----------------------------------------------------------------------------------
 # Keep-or-drop block-sparse attention  ([BSA] §3.3, §4.3)
 # ----------------------------------------------------------------------------------
-def keep_or_drop_head(q, k, v, row_ptr, col_idx, block, scale, qblocks=None):
-    """O_i = softmax(s Q_i K_{S_i}^T) V_{S_i}, the softmax taken over S_i only.
+def keep_or_drop_head(q, k, v, row_ptr, col_idx, block, scale, qblocks=None, key_valid=None):
+    """O_i = softmax(s Q_i K_{S_i}^T) V_{S_i}, the softmax taken over S_i only (over the
+    real keys of S_i when ``key_valid`` marks padding).
 
     Returns (out [n, d], lse [n]) for the rows of the requested query blocks (all by
     default), in block order.
@@ -114,6 +135,7 @@ def keep_or_drop_head(q, k, v, row_ptr, col_idx, block, scale, qblocks=None):
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     L, d = q.shape
     M = L // block
+    valid = _valid(key_valid, M, block)
     blocks = range(M) if qblocks is None else qblocks
     outs, lses = [], []
     for i in blocks:
@@ -123,8 +145,8 @@ def keep_or_drop_head(q, k, v, row_ptr, col_idx, block, scale, qblocks=None):
             outs.append(np.zeros((block, v.shape[1])))
             lses.append(np.full(block, -np.inf))
             continue
-        idx = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel])
-        a = scale * (qi @ k[idx].T)                       # [B, |S_i| B]
+        idx = _keys(sel, block, valid)
+        a = scale * (qi @ k[idx].T)                       # [B, real keys of S_i]
         m = a.max(axis=1, keepdims=True)
         p = np.exp(a - m)
         den = p.sum(axis=1)
@@ -136,24 +158,26 @@ def keep_or_drop_head(q, k, v, row_ptr, col_idx, block, scale, qblocks=None):
 # ----------------------------------------------------------------------------------
 # a2. Per-block statistics  ([PISA] §2: centroids, value sums, H_j, H-bar, M_j)
 # ----------------------------------------------------------------------------------
-def precompute_head(k, v, block):
+def precompute_head(k, v, block, key_valid=None):
     """Return kbar [M,d], vsum [M,d], H [M,d,d], Hbar [d,d], Mnorm [M].
 
-    kbar_j = (1/B) sum_n k_{j,n};  vsum_j = sum_n v_{j,n};
+    kbar_j = (1/B_j) sum_n k_{j,n};  vsum_j = sum_n v_{j,n};
     H_j = sum_n (k_{j,n} - kbar_j)^T v_{j,n}  (centred form, d_k rows x d_v cols);
     Hbar = (1/M) sum_j H_j;  Mnorm_j = ||H_j - Hbar||_F.
+    The sums run over the B_j real tokens of block j (B_j = B without padding).
     """
     k, v = (np.asarray(x, dtype=np.float64) for x in (k, v))
     L, d = k.shape
     M = L // block
+    valid = _valid(key_valid, M, block)
     kb = k.reshape(M, block, d)
     vb = v.reshape(M, block, v.shape[1])
-    kbar = kb.mean(axis=1)
-    vsum = vb.sum(axis=1)
+    kbar = np.stack([kb[j, :valid[j]].mean(axis=0) for j in range(M)])
+    vsum = np.stack([vb[j, :valid[j]].sum(axis=0) for j in range(M)])
     H = np.empty((M, d, v.shape[1]))
     for j in range(M):
-        centred = kb[j] - kbar[j]
-        H[j] = centred.T @ vb[j]
+        centred = kb[j, :valid[j]] - kbar[j]
+        H[j] = centred.T @ vb[j, :valid[j]]
     Hbar = H.mean(axis=0)
     Mnorm = np.sqrt(((H - Hbar) ** 2).sum(axis=(1, 2)))
     return kbar, vsum, H, Hbar, Mnorm
@@ -162,20 +186,25 @@ def precompute_head(k, v, block):
 # ----------------------------------------------------------------------------------
 # a3. Covariance-aware top-k routing  ([PISA] §2 covariance-aware routing)
 # ----------------------------------------------------------------------------------
-def route_head(q, kbar, Mnorm, block, k_top, lam, scale):
+def route_head(q, kbar, Mnorm, block, k_top, lam, scale, key_valid=None):
     """Top-k KV blocks per query block; returns (row_ptr, col_idx, scores [M, M]).
 
-    qbar_i = mean of the B queries of block i; p_ij = softmax_j(s qbar_i . kbar_j);
+    qbar_i = mean of the real queries of block i; p_ij = softmax_j(s qbar_i . kbar_j);
     score_ij = p_ij + lam * Mnorm_j / sum_j' Mnorm_j' (second term 0 if the sum is 0).
-    S_i = the k_top largest scores, ties broken towards the smaller j; the list is
-    emitted in ascending j.
+    S_i = the padded blocks (every row), then the largest scores up to k_top, ties
+    broken towards the smaller j; the list is emitted in ascending j.
     """
     q = np.asarray(q, dtype=np.float64)
     kbar = np.asarray(kbar, dtype=np.float64)
     Mnorm = np.asarray(Mnorm, dtype=np.float64)
     L, d = q.shape
     M = L // block
-    qbar = q.reshape(M, block, d).mean(axis=1)
+    valid = _valid(key_valid, M, block)
+    forced = [j for j in range(M) if valid[j] < block]
+    if len(forced) > k_top:
+        raise ValueError("k_top is smaller than the number of padded blocks")
+    qb = q.reshape(M, block, d)
+    qbar = np.stack([qb[i, :valid[i]].mean(axis=0) for i in range(M)])
     a = scale * (qbar @ kbar.T)                           # [M, M]
     p = np.exp(a - a.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
@@ -185,8 +214,8 @@ def route_head(q, kbar, Mnorm, block, k_top, lam, scale):
     row_ptr = np.arange(M + 1, dtype=np.int32) * k_top
     col_idx = np.empty(M * k_top, dtype=np.int32)
     for i in range(M):
-        order = sorted(range(M), key=lambda j: (-scores[i, j], j))
-        col_idx[i * k_top:(i + 1) * k_top] = sorted(order[:k_top])
+        order = sorted((j for j in range(M) if j not in forced), key=lambda j: (-scores[i, j], j))
+        col_idx[i * k_top:(i + 1) * k_top] = sorted(forced + order[:k_top - len(forced)])
     return row_ptr, col_idx, scores
 
 
@@ -194,15 +223,17 @@ def route_head(q, kbar, Mnorm, block, k_top, lam, scale):
 # a4-a6. Piecewise sparse attention  ([PISA] §2: o_t = N_t / D_t)
 # ----------------------------------------------------------------------------------
 def pisa_head(q, k, v, row_ptr, col_idx, block, scale, kbar, vsum, Hbar,
-              qblocks=None, Hblocks=None):
+              qblocks=None, Hblocks=None, key_valid=None):
     """Exact terms over S_i, zeroth-order centroid terms and the first-order
     correction over U_i, inside one normalisation.
 
     N_t = sum_{j in S_i} sum_n e^{s q_t.k_{j,n} - m_t} v_{j,n}
           + sum_{j in U_i} alpha_tj vsum_j
           + s (q_t Hbar) sum_{j in U_i} alpha_tj
-    D_t = sum_{j in S_i} sum_n e^{s q_t.k_{j,n} - m_t} + sum_{j in U_i} B alpha_tj
+    D_t = sum_{j in S_i} sum_n e^{s q_t.k_{j,n} - m_t} + sum_{j in U_i} B_j alpha_tj
     alpha_tj = e^{s q_t.kbar_j - m_t};  o_t = N_t / D_t.
+    B_j is the block's number of real tokens (B without padding); the exact sums run
+    over real keys only.
 
     With ``Hblocks`` ([M, d, d]) the first-order term uses each block's own H_j,
     s alpha_tj (q_t H_j), instead of the shared Hbar: the per-block variant that the
@@ -213,6 +244,7 @@ def pisa_head(q, k, v, row_ptr, col_idx, block, scale, kbar, vsum, Hbar,
     kbar, vsum, Hbar = (np.asarray(x, dtype=np.float64) for x in (kbar, vsum, Hbar))
     L, d = q.shape
     M = L // block
+    valid = _valid(key_valid, M, block)
     blocks = range(M) if qblocks is None else qblocks
     outs, lses = [], []
     for i in blocks:
@@ -220,8 +252,8 @@ def pisa_head(q, k, v, row_ptr, col_idx, block, scale, kbar, vsum, Hbar,
         sel = _row(row_ptr, col_idx, i)
         uns = [j for j in range(M) if j not in set(sel)]
         if sel:
-            idx = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel])
-            a_ex = scale * (qi @ k[idx].T)                # exact scores [B, |S_i| B]
+            idx = _keys(sel, block, valid)
+            a_ex = scale * (qi @ k[idx].T)                # exact scores [B, real keys]
         else:
             idx = np.zeros(0, dtype=np.int64)
             a_ex = np.zeros((block, 0))
@@ -239,7 +271,7 @@ def pisa_head(q, k, v, row_ptr, col_idx, block, scale, kbar, vsum, Hbar,
         else:
             for c, j in enumerate(uns):
                 num += scale * alpha[:, c:c + 1] * (qi @ Hblocks[j])
-        den = p.sum(axis=1) + block * alpha.sum(axis=1)
+        den = p.sum(axis=1) + alpha @ np.asarray([valid[j] for j in uns], dtype=np.float64)
         outs.append(num / den[:, None])
         lses.append(m + np.log(den))
     return np.concatenate(outs), np.concatenate(lses)
@@ -261,20 +293,20 @@ def _bh(x):
     return x.reshape(-1, x.shape[-2], x.shape[-1])
 
 
-def precompute(k, v, block):
+def precompute(k, v, block, key_valid=None):
     """Apply precompute_head to every (batch, head); arrays stacked on axis 0."""
-    res = [precompute_head(kk, vv, block) for kk, vv in zip(_bh(k), _bh(v))]
+    res = [precompute_head(kk, vv, block, key_valid) for kk, vv in zip(_bh(k), _bh(v))]
     return tuple(np.stack([r[n] for r in res]) for n in range(5))
 
 
-def route(q, kbar, Mnorm, block, k_top, lam, scale):
+def route(q, kbar, Mnorm, block, k_top, lam, scale, key_valid=None):
     """Per-head routing. row_ptr is [heads, M+1] (flattened) holding absolute offsets
     into the stacked col_idx; head h's lists start at h * M * k_top."""
     qs = _bh(q)
     M = qs.shape[1] // block
     rps, cis, scs = [], [], []
     for h, qq in enumerate(qs):
-        rp, ci, sc = route_head(qq, kbar[h], Mnorm[h], block, k_top, lam, scale)
+        rp, ci, sc = route_head(qq, kbar[h], Mnorm[h], block, k_top, lam, scale, key_valid)
         rps.append(rp + h * M * k_top)
         cis.append(ci)
         scs.append(sc)

@@ -350,3 +350,130 @@ def test_batched_route_csr_layout():
         hrp, hci = orc.head_csr(rp, ci, h, M, True)
         rp1, ci1, _ = orc.route_head(q[h], kbar[h], Mn[h], block, 2, 1.0, 0.5)
         assert hrp.tolist() == rp1.tolist() and hci.tolist() == ci1.tolist()
+
+
+# ------------------------------------------------------------- token-level padding
+def _padded_case(seed, M=6, block=8, d=8):
+    """A head whose blocks 0 and 3 carry padding at their tail (a text segment padded
+    to the block size, and a one-token timestep block)."""
+    r = _rng(seed)
+    q, k, v = r.standard_normal((3, M * block, d))
+    valid = [block] * M
+    valid[0], valid[3] = 5, 1
+    return q, k, v, valid, block
+
+
+def _garbage(x, valid, block, seed):
+    """The same tensor with every padded row replaced by large random values."""
+    y = np.array(x, copy=True)
+    r = _rng(seed)
+    for j, n in enumerate(valid):
+        y[j * block + n:(j + 1) * block] = 1e3 * r.standard_normal((block - n, y.shape[1]))
+    return y
+
+
+def _masked_sdpa(q, k, v, scale, allowed):
+    """torch float64 scaled_dot_product_attention with a boolean key mask."""
+    qt, kt, vt = (torch.from_numpy(np.asarray(x, dtype=np.float64))[None, None]
+                  for x in (q, k, v))
+    m = torch.from_numpy(allowed)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=m,
+                                                            scale=scale)[0, 0].numpy()
+
+
+def test_padding_with_full_blocks_changes_nothing():
+    q, k, v, _, block = _padded_case(20)
+    M = q.shape[0] // block
+    full = [block] * M
+    s = 1 / math.sqrt(q.shape[1])
+    rp, ci = _random_csr(M, 3, 21)
+    a = orc.precompute_head(k, v, block)
+    b_ = orc.precompute_head(k, v, block, key_valid=full)
+    for x, y in zip(a, b_):
+        np.testing.assert_array_equal(x, y)
+    np.testing.assert_array_equal(orc.keep_or_drop_head(q, k, v, rp, ci, block, s)[0],
+                                  orc.keep_or_drop_head(q, k, v, rp, ci, block, s, key_valid=full)[0])
+    kbar, vsum, H, Hbar, Mn = a
+    np.testing.assert_array_equal(
+        orc.pisa_head(q, k, v, rp, ci, block, s, kbar, vsum, Hbar)[0],
+        orc.pisa_head(q, k, v, rp, ci, block, s, kbar, vsum, Hbar, key_valid=full)[0])
+    np.testing.assert_array_equal(orc.route_head(q, kbar, Mn, block, 2, 1.0, s)[1],
+                                  orc.route_head(q, kbar, Mn, block, 2, 1.0, s, key_valid=full)[1])
+
+
+def test_padded_rows_do_not_matter():
+    """Nothing computed for real tokens depends on what the padded positions hold."""
+    q, k, v, valid, block = _padded_case(22)
+    M = q.shape[0] // block
+    s = 1 / math.sqrt(q.shape[1])
+    q2, k2, v2 = (_garbage(x, valid, block, 23 + n) for n, x in enumerate((q, k, v)))
+    st1 = orc.precompute_head(k, v, block, key_valid=valid)
+    st2 = orc.precompute_head(k2, v2, block, key_valid=valid)
+    for x, y in zip(st1, st2):
+        np.testing.assert_allclose(x, y, rtol=1e-12, atol=1e-12)
+    kbar, vsum, H, Hbar, Mn = st1
+    rp1, ci1, sc1 = orc.route_head(q, kbar, Mn, block, 3, 1.0, s, key_valid=valid)
+    rp2, ci2, sc2 = orc.route_head(q2, kbar, Mn, block, 3, 1.0, s, key_valid=valid)
+    np.testing.assert_array_equal(ci1, ci2)
+    np.testing.assert_allclose(sc1, sc2, rtol=1e-12, atol=1e-12)
+    real = np.concatenate([np.arange(j * block, j * block + valid[j]) for j in range(M)])
+    o1, _ = orc.pisa_head(q, k, v, rp1, ci1, block, s, kbar, vsum, Hbar, key_valid=valid)
+    o2, _ = orc.pisa_head(q2, k2, v2, rp1, ci1, block, s, kbar, vsum, Hbar, key_valid=valid)
+    np.testing.assert_allclose(o1[real], o2[real], rtol=1e-12, atol=1e-12)
+    o1, _ = orc.keep_or_drop_head(q, k, v, rp1, ci1, block, s, key_valid=valid)
+    o2, _ = orc.keep_or_drop_head(q2, k2, v2, rp1, ci1, block, s, key_valid=valid)
+    np.testing.assert_allclose(o1[real], o2[real], rtol=1e-12, atol=1e-12)
+
+
+def test_keep_or_drop_with_padding_is_masked_sdpa():
+    q, k, v, valid, block = _padded_case(24)
+    M = q.shape[0] // block
+    s = 1 / math.sqrt(q.shape[1])
+    rp, ci = _random_csr(M, 3, 25)
+    out, _ = orc.keep_or_drop_head(q, k, v, rp, ci, block, s, key_valid=valid)
+    allowed = np.zeros((q.shape[0], q.shape[0]), dtype=bool)
+    for i in range(M):
+        for j in ci[rp[i]:rp[i + 1]]:
+            allowed[i * block:(i + 1) * block, j * block:j * block + valid[j]] = True
+    np.testing.assert_allclose(out, _masked_sdpa(q, k, v, s, allowed), rtol=1e-10, atol=1e-12)
+
+
+def test_pisa_full_selection_with_padding_is_masked_dense():
+    q, k, v, valid, block = _padded_case(26)
+    M = q.shape[0] // block
+    s = 1 / math.sqrt(q.shape[1])
+    rp, ci = orc.dense_to_csr(np.ones((M, M), dtype=bool))
+    kbar, vsum, H, Hbar, Mn = orc.precompute_head(k, v, block, key_valid=valid)
+    out, lse = orc.pisa_head(q, k, v, rp, ci, block, s, kbar, vsum, Hbar, key_valid=valid)
+    allowed = np.zeros((q.shape[0], q.shape[0]), dtype=bool)
+    for j in range(M):
+        allowed[:, j * block:j * block + valid[j]] = True
+    np.testing.assert_allclose(out, _masked_sdpa(q, k, v, s, allowed), rtol=1e-10, atol=1e-12)
+
+
+def test_padded_block_statistics_use_real_tokens_only():
+    """A block whose real keys are all one vector c (padding holds other values) has
+    centroid c and H_j = 0; its value sum counts the real rows only."""
+    q, k, v, valid, block = _padded_case(27)
+    c = _rng(28).standard_normal(k.shape[1])
+    k = np.array(k, copy=True)
+    k[0:valid[0]] = c
+    kbar, vsum, H, Hbar, Mn = orc.precompute_head(k, v, block, key_valid=valid)
+    np.testing.assert_allclose(kbar[0], c, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(H[0], 0.0, atol=1e-12)
+    np.testing.assert_allclose(vsum[0], np.asarray(v)[0:valid[0]].sum(axis=0), rtol=1e-13)
+    np.testing.assert_allclose(kbar[3], k[3 * block], rtol=1e-13)   # the one-token block
+
+
+def test_routing_places_every_padded_block_in_every_list():
+    q, k, v, valid, block = _padded_case(29)
+    M = q.shape[0] // block
+    s = 1 / math.sqrt(q.shape[1])
+    kbar, vsum, H, Hbar, Mn = orc.precompute_head(k, v, block, key_valid=valid)
+    for kk in (2, 4):
+        rp, ci, sc = orc.route_head(q, kbar, Mn, block, kk, 1.0, s, key_valid=valid)
+        for i in range(M):
+            row = list(ci[rp[i]:rp[i + 1]])
+            assert 0 in row and 3 in row and row == sorted(row) and len(row) == kk
+    with pytest.raises(ValueError):
+        orc.route_head(q, kbar, Mn, block, 1, 1.0, s, key_valid=valid)
