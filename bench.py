@@ -53,6 +53,14 @@ def forward_flops(w, k_top: int, mode: str, row_lens=None) -> float:
     return w.batch * w.heads * total
 
 
+GENERATOR_TEXT = {
+    "iid": "N(0,1)",
+    "block_centres": "K = per-block centre + 0.5 N(0,1), V = N(0,1)",
+    "field2d_hot": "smooth 2-D field + 0.3 N(0,1), 4 hot blocks x3",
+    "field3d": "smooth 3-D field + 0.3 N(0,1)",
+}
+
+
 def needs_precompute(w) -> bool:
     """The statistics feed the routing and PISA's Taylor tail; a fixed mask in the other
     modes needs neither."""
@@ -243,23 +251,25 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
     q, k, v = synth.make_qkv(w, seed=seed, heads=heads)
     scale = 1 / math.sqrt(w.head_dim)
     fixed = orc.dense_to_csr(orc.mask_dense(**w.mask)) if w.mask else None
+    kv = w.valid_tokens()
     t0 = time.perf_counter()
     for h in heads:
         qf, kf, vf = (x[h].to(torch.float64).numpy() for x in (q, k, v))
         if fixed is not None and w.mode == "keep_or_drop":
-            orc.keep_or_drop_head(qf, kf, vf, fixed[0], fixed[1], w.block, scale)
+            orc.keep_or_drop_head(qf, kf, vf, fixed[0], fixed[1], w.block, scale, key_valid=kv)
             continue
-        kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block)
+        kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block, kv)
         if fixed is not None:
             rp, ci = fixed
         else:
-            rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale)
+            rp, ci, _ = orc.route_head(qf, kbar, Mn, w.block, k_top, LAMBDA, scale, kv)
         if w.mode == "pisa":
-            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar)
+            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar, key_valid=kv)
         elif w.mode == "pisa_block":
-            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar, Hblocks=H)
+            orc.pisa_head(qf, kf, vf, rp, ci, w.block, scale, kbar, vsum, Hbar, Hblocks=H,
+                          key_valid=kv)
         else:
-            orc.keep_or_drop_head(qf, kf, vf, rp, ci, w.block, scale)
+            orc.keep_or_drop_head(qf, kf, vf, rp, ci, w.block, scale, key_valid=kv)
     dt = time.perf_counter() - t0
     BH = w.batch * w.heads
     return {"seconds_sample": dt, "seconds_full_est": dt * BH / len(heads), "cores": threads,
@@ -279,6 +289,9 @@ def run_ours(args, w, world, rank, local):
     q, k, v = synth.make_qkv(w, seed=args.seed + rank)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
+    # real tokens per block (token padding), a constant of the workload like its mask
+    kv = None if not w.key_valid else torch.tensor(w.valid_tokens(), dtype=torch.int32,
+                                                   device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     stats = dict(kbar=torch.empty(BH, M, d, **f32), vsum=torch.empty(BH, M, d, **f32),
                  Hbar=torch.empty(BH, d, d, **f32), Mnorm=torch.empty(BH, M, **f32))
@@ -305,16 +318,16 @@ def run_ours(args, w, world, rank, local):
             ev[0].record(stream)
         if needs_precompute(w):
             b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
-                             stats["Mnorm"], None, ws_p, st)
+                             stats["Mnorm"], None, ws_p, st, key_valid=kv)
         if ev:
             ev[1].record(stream)
         if not w.mask:
             b.bsa_route(qx, stats["kbar"], stats["Mnorm"], w.block, k_top, LAMBDA, 0.0, rp, ci,
-                        None, st)
+                        None, st, key_valid=kv)
         if ev:
             ev[2].record(stream)
         b.bsa_forward(qx, kx, vx, w.block, rp, ci, per_head, mode, stats["kbar"],
-                      stats["vsum"], stats["Hbar"], 0.0, O, None, ws_f, st)
+                      stats["vsum"], stats["Hbar"], 0.0, O, None, ws_f, st, key_valid=kv)
         if ev:
             ev[3].record(stream)
 
@@ -391,11 +404,12 @@ def run_ours(args, w, world, rank, local):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded: Q ~ N(0,1); K, V = smooth 3-D field + 0.3 N(0,1))",
+        "data": "synthetic (seeded: Q ~ N(0,1); K, V: " + GENERATOR_TEXT[w.generator] + ")",
         "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": L,
                    "head_dim": d, "block": w.block, "mode": w.mode, "density": w.density,
                    "k_top": None if w.mask else k_top, "lambda": LAMBDA,
                    "lists": "fixed multimodal mask (shared)" if w.mask else "bsa_route top-k",
+                   "real_tokens_per_block": w.valid_tokens() if w.key_valid else None,
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2 (Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB)"},
         "forward_ms": round(fwd_ms, 4), "forward_tflops": round(achieved, 3),

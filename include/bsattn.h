@@ -31,6 +31,16 @@
  *     inputs were found malformed leaves its outputs unwritten.
  *   - Supported: d in {64, 128}; block in {64, 128}; L % block == 0; M <= 2048.
  *     Anything else returns BSA_ERR_UNSUPPORTED.
+ *   - Token padding ([BSA] §4.1 pads the text segment to a multiple of the block size;
+ *     §7.3 gives a timestep token its own block): `key_valid` (nullable, device int32
+ *     [M], shared by every (batch, head)) is the number of leading real tokens of each
+ *     block, 1..block; the rest of the block is padding. NULL means no padding. Padded
+ *     keys receive no attention weight; centroids, value sums, H_j and pooled queries
+ *     are taken over real tokens only; an unselected block's Taylor-tail weight is its
+ *     real-token count; a padded block is always computed exactly: bsa_route places it
+ *     in every list, and bsa_forward in the PISA modes reports BSA_ERR_BAD_PADDING for a
+ *     list that lacks one. Padded query rows are computed like any other row. Values
+ *     outside 1..block report BSA_ERR_BAD_PADDING (and are clamped).
  */
 #ifndef BSATTN_H
 #define BSATTN_H
@@ -57,8 +67,10 @@ typedef enum {
   BSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (device-detected) */
   BSA_ERR_WORKSPACE = 6,     /* workspace null or smaller than bsa_workspace_bytes   */
   BSA_ERR_CAPACITY = 7,      /* an output list would exceed its capacity (device)    */
-  BSA_ERR_SCRATCH_LIMIT = 8  /* bsa_forward_noalloc: the shape needs more scratch than
+  BSA_ERR_SCRATCH_LIMIT = 8, /* bsa_forward_noalloc: the shape needs more scratch than
                                 BSA_NOALLOC_SCRATCH_BYTES                            */
+  BSA_ERR_BAD_PADDING = 9    /* key_valid out of range, or a padded block missing from a
+                                PISA list (device-detected)                          */
 } bsa_status;
 
 /* Size of the device scratch array built into the library for bsa_forward_noalloc. */
@@ -127,24 +139,27 @@ BSA_API bsa_status bsa_build_mask(const bsa_mask_desc* desc, int32_t* row_ptr, i
                           int64_t col_capacity, int32_t* status, void* stream);
 
 /* bsa_precompute — per-block statistics of [PISA] §2 ("precompute" stage):
- *   kbar_j = (1/B) sum_n k_{j,n}                     -> kbar  fp32 [BH, M, d]
+ *   kbar_j = (1/B_j) sum_n k_{j,n}                   -> kbar  fp32 [BH, M, d]
  *   vsum_j = sum_n v_{j,n}                           -> vsum  fp32 [BH, M, d]
  *   H_j    = sum_n (k_{j,n} - kbar_j)^T v_{j,n}      (d_k rows x d_v cols)
  *   Hbar   = (1/M) sum_j H_j  (mean over all blocks of the head) -> Hbar fp32 [BH, d, d]
  *   Mnorm_j = ||H_j - Hbar||_F (Frobenius)           -> Mnorm fp32 [BH, M]
  *   Hblk (nullable) receives every H_j              -> fp32 [BH, M, d, d]
+ *   (sums over the B_j real tokens of block j: B_j = key_valid[j], or B)
  * K, V are bf16 [Bt, H, L, d]. workspace: device, >= bsa_workspace_bytes(
  * BSA_CALL_PRECOMPUTE, ...) bytes, contents scratch. */
 BSA_API bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int32_t H, int32_t L,
-                          int32_t d, int32_t block, float* kbar, float* vsum, float* Hbar,
-                          float* Mnorm, float* Hblk, void* workspace, size_t ws_bytes,
-                          int32_t* status, void* stream);
+                          int32_t d, int32_t block, const int32_t* key_valid, float* kbar,
+                          float* vsum, float* Hbar, float* Mnorm, float* Hblk,
+                          void* workspace, size_t ws_bytes, int32_t* status, void* stream);
 
 /* bsa_route — covariance-aware top-k block selection ([PISA] §2, routing).
- *   qbar_i   = mean of the B queries of block i;
+ *   qbar_i   = mean of the (real) queries of block i;
  *   p_ij     = softmax_j(scale * qbar_i . kbar_j) over all M key blocks;
  *   score_ij = p_ij + lambda * Mnorm_j / sum_j' Mnorm_j'  (term is 0 if the sum is 0);
- *   S_i      = the k_top highest scores, ties to the smaller j, written ascending.
+ *   S_i      = the padded blocks, then the highest scores up to k_top, ties to the
+ *              smaller j, written ascending (BSA_ERR_BAD_PADDING if k_top is smaller
+ *              than the number of padded blocks).
  * (The pages say the score "combines" the attention score with M_j without a
  * formula; this mix of two distributions is this library's reading.)
  *   Q        bf16 [Bt, H, L, d];  kbar fp32 [BH, M, d];  Mnorm fp32 [BH, M];
@@ -155,9 +170,9 @@ BSA_API bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int3
  *   scores   nullable fp32 [BH, M, M] receives score_ij.
  * 1 <= k_top <= M. */
 BSA_API bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32_t Bt,
-                     int32_t H, int32_t L, int32_t d, int32_t block, int32_t k_top,
-                     float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
-                     float* scores, int32_t* status, void* stream);
+                     int32_t H, int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
+                     int32_t k_top, float lambda, float scale, int32_t* row_ptr,
+                     int32_t* col_idx, float* scores, int32_t* status, void* stream);
 
 /* bsa_forward — fused online-softmax attention over block lists.
  *   mode BSA_MODE_KEEP_OR_DROP ([BSA] §3.3):
@@ -188,9 +203,13 @@ BSA_API bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnor
  *   scale        0 selects 1/sqrt(d);
  *   lse          nullable fp32 [BH, L]: natural-log denominator, m_t + log D_t;
  *   workspace    device, >= bsa_workspace_bytes(BSA_CALL_FORWARD, ...) bytes.
- * Malformed lists set BSA_ERR_BAD_CSR in *status and leave O unwritten. */
+ *   key_valid    see the conventions: padded keys are masked; in the PISA modes every
+ *                padded block must be in every list.
+ * Malformed lists set BSA_ERR_BAD_CSR (a missing padded block BSA_ERR_BAD_PADDING) in
+ * *status and leave O unwritten. */
 BSA_API bsa_status bsa_forward(const void* Q, const void* K, const void* V, int32_t Bt, int32_t H,
-                       int32_t L, int32_t d, int32_t block, const int32_t* row_ptr,
+                       int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
+                       const int32_t* row_ptr,
                        const int32_t* col_idx, int64_t nnz_total, int32_t csr_per_head,
                        int32_t mode, const float* kbar, const float* vsum,
                        const float* Hbar, float scale, void* O, float* lse,
@@ -216,7 +235,8 @@ BSA_API bsa_status bsa_forward(const void* Q, const void* K, const void* V, int3
  *     each term rounded up to 256), the other modes 256 bytes. Other errors as bsa_forward. */
 BSA_API bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void* V, int32_t Bt,
                                        int32_t H, int32_t L, int32_t d, int32_t block,
-                                       const int32_t* row_ptr, const int32_t* col_idx,
+                                       const int32_t* key_valid, const int32_t* row_ptr,
+                                       const int32_t* col_idx,
                                        int64_t nnz_total, int32_t csr_per_head, int32_t mode,
                                        const float* kbar, const float* vsum, const float* Hbar,
                                        float scale, void* O, float* lse, int32_t* status,

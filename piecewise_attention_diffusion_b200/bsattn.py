@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsattn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_BAD_CSR, ERR_TIMEOUT, ERR_WORKSPACE, \
-    ERR_CAPACITY, ERR_SCRATCH_LIMIT = range(9)
+    ERR_CAPACITY, ERR_SCRATCH_LIMIT, ERR_BAD_PADDING = range(10)
 NOALLOC_SCRATCH_BYTES = 16 << 20
 MODE_KEEP_OR_DROP, MODE_PISA, MODE_PISA_BLOCK = 0, 1, 2
 CALL_BUILD_MASK, CALL_PRECOMPUTE, CALL_ROUTE, CALL_FORWARD = 0, 1, 2, 3
@@ -54,13 +54,13 @@ _SIGS = {
     "bsa_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "bsa_build_mask": (_i32, [ctypes.POINTER(MaskDesc), _vp, _vp, _i64, _vp, _vp]),
     "bsa_precompute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp,
-                              _vp, _sz, _vp, _vp]),
-    "bsa_route": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _f32, _vp,
-                         _vp, _vp, _vp, _vp]),
-    "bsa_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _i32,
-                           _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
-    "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i64,
-                                   _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp]),
+                              _vp, _vp, _sz, _vp, _vp]),
+    "bsa_route": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _f32, _f32,
+                         _vp, _vp, _vp, _vp, _vp]),
+    "bsa_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i64,
+                           _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
+                                   _i64, _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp]),
     "bsa_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
 }
 
@@ -152,8 +152,15 @@ def _bhld(x, name):
     return x.shape
 
 
+def _key_valid(key_valid, L, block):
+    """Check the per-block real-token counts (int32[L/block], shared by all heads)."""
+    if key_valid is not None:
+        _need(key_valid, torch.int32, "key_valid", (L // block,))
+    return _ptr(key_valid)
+
+
 def bsa_precompute(K, V, block, kbar, vsum, Hbar, Mnorm, Hblk=None, workspace=None,
-                   status=None, stream=None):
+                   status=None, stream=None, key_valid=None):
     Bt, H, L, d = _bhld(K, "K")
     _need(V, torch.bfloat16, "V", K.shape)
     M = L // block
@@ -164,13 +171,14 @@ def bsa_precompute(K, V, block, kbar, vsum, Hbar, Mnorm, Hblk=None, workspace=No
     if Hblk is not None:
         _need(Hblk, torch.float32, "Hblk", (Bt * H, M, d, d))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().bsa_precompute(_ptr(K), _ptr(V), Bt, H, L, d, block, _ptr(kbar), _ptr(vsum),
+    _check(lib().bsa_precompute(_ptr(K), _ptr(V), Bt, H, L, d, block,
+                                _key_valid(key_valid, L, block), _ptr(kbar), _ptr(vsum),
                                 _ptr(Hbar), _ptr(Mnorm), _ptr(Hblk), _ptr(workspace), ws_bytes,
                                 _ptr(status), _stream(stream)), "bsa_precompute")
 
 
 def bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores=None,
-              status=None, stream=None):
+              status=None, stream=None, key_valid=None):
     Bt, H, L, d = _bhld(Q, "Q")
     M = L // block
     _need(kbar, torch.float32, "kbar", (Bt * H, M, d))
@@ -179,13 +187,14 @@ def bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores
     _need(col_idx, torch.int32, "col_idx", (Bt * H * M * k_top,))
     if scores is not None:
         _need(scores, torch.float32, "scores", (Bt * H, M, M))
-    _check(lib().bsa_route(_ptr(Q), _ptr(kbar), _ptr(Mnorm), Bt, H, L, d, block, k_top,
+    _check(lib().bsa_route(_ptr(Q), _ptr(kbar), _ptr(Mnorm), Bt, H, L, d, block,
+                           _key_valid(key_valid, L, block), k_top,
                            float(lam), float(scale), _ptr(row_ptr), _ptr(col_idx),
                            _ptr(scores), _ptr(status), _stream(stream)), "bsa_route")
 
 
 def bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum, Hbar, scale,
-                O, lse=None, workspace=None, status=None, stream=None):
+                O, lse=None, workspace=None, status=None, stream=None, key_valid=None):
     Bt, H, L, d = _bhld(Q, "Q")
     _need(K, torch.bfloat16, "K", Q.shape)
     _need(V, torch.bfloat16, "V", Q.shape)
@@ -200,15 +209,15 @@ def bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum
     if lse is not None:
         _need(lse, torch.float32, "lse", (Bt * H, L))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().bsa_forward(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block, _ptr(row_ptr),
-                             _ptr(col_idx), col_idx.numel(), int(csr_per_head), int(mode),
+    _check(lib().bsa_forward(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block,
+                             _key_valid(key_valid, L, block), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), int(csr_per_head), int(mode),
                              _ptr(kbar), _ptr(vsum), _ptr(Hbar), float(scale), _ptr(O),
                              _ptr(lse), _ptr(workspace), ws_bytes, _ptr(status),
                              _stream(stream)), "bsa_forward")
 
 
 def bsa_forward_noalloc(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum, Hbar,
-                        scale, O, lse=None, status=None, stream=None):
+                        scale, O, lse=None, status=None, stream=None, key_valid=None):
     """bsa_forward without a workspace argument: the library's built-in device scratch
     array is used instead, for callers that cannot allocate device memory."""
     Bt, H, L, d = _bhld(Q, "Q")
@@ -225,7 +234,7 @@ def bsa_forward_noalloc(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kb
     if lse is not None:
         _need(lse, torch.float32, "lse", (Bt * H, L))
     _check(lib().bsa_forward_noalloc(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block,
-                                     _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                     _key_valid(key_valid, L, block), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
                                      int(csr_per_head), int(mode), _ptr(kbar), _ptr(vsum),
                                      _ptr(Hbar), float(scale), _ptr(O), _ptr(lse),
                                      _ptr(status), _stream(stream)), "bsa_forward_noalloc")
@@ -257,7 +266,7 @@ def build_mask(desc, device="cuda", status=None):
     return row_ptr, col_idx[:nnz].clone()
 
 
-def precompute(K, V, block, want_blocks=False, status=None, ws=None):
+def precompute(K, V, block, want_blocks=False, status=None, ws=None, key_valid=None):
     Bt, H, L, d = K.shape
     BH, M = Bt * H, L // block
     f = dict(dtype=torch.float32, device=K.device)
@@ -267,23 +276,25 @@ def precompute(K, V, block, want_blocks=False, status=None, ws=None):
     if ws is None:
         ws = workspace(CALL_PRECOMPUTE, Bt, H, L, d, block, K.device)
     bsa_precompute(K, V, block, out["kbar"], out["vsum"], out["Hbar"], out["Mnorm"],
-                   out["Hblk"], ws, status)
+                   out["Hblk"], ws, status, key_valid=key_valid)
     return out
 
 
-def route(Q, kbar, Mnorm, block, k_top, lam=1.0, scale=0.0, want_scores=False, status=None):
+def route(Q, kbar, Mnorm, block, k_top, lam=1.0, scale=0.0, want_scores=False, status=None,
+          key_valid=None):
     Bt, H, L, d = Q.shape
     BH, M = Bt * H, L // block
     row_ptr = torch.empty(BH * (M + 1), dtype=torch.int32, device=Q.device)
     col_idx = torch.empty(BH * M * k_top, dtype=torch.int32, device=Q.device)
     scores = torch.empty(BH, M, M, dtype=torch.float32, device=Q.device) if want_scores \
         else None
-    bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores, status)
+    bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores, status,
+              key_valid=key_valid)
     return row_ptr, col_idx, scores
 
 
 def forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, stats=None, scale=0.0,
-            want_lse=False, status=None, ws=None, out=None):
+            want_lse=False, status=None, ws=None, out=None, key_valid=None):
     Bt, H, L, d = Q.shape
     O = torch.empty_like(Q) if out is None else out
     lse = torch.empty(Bt * H, L, dtype=torch.float32, device=Q.device) if want_lse else None
@@ -291,7 +302,7 @@ def forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, stats=None, sc
         ws = workspace(CALL_FORWARD, Bt, H, L, d, block, Q.device)
     st = stats or {}
     bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, st.get("kbar"),
-                st.get("vsum"), st.get("Hbar"), scale, O, lse, ws, status)
+                st.get("vsum"), st.get("Hbar"), scale, O, lse, ws, status, key_valid=key_valid)
     return O, lse
 
 

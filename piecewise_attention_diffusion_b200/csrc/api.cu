@@ -23,6 +23,7 @@ bsa_status check_shape(const Shape& s) {
   if (s.M() > kMaxBlocks) return BSA_ERR_UNSUPPORTED;
   if ((int64_t)s.Bt * s.H * s.L * s.d >= (int64_t)1 << 40) return BSA_ERR_UNSUPPORTED;
   if ((int64_t)s.Bt * s.H > 65535) return BSA_ERR_UNSUPPORTED;  // grid.y limit
+  if ((reinterpret_cast<uintptr_t>(s.key_valid) & 3u) != 0) return BSA_ERR_INVALID_ARG;
   return BSA_OK;
 }
 
@@ -43,7 +44,7 @@ int mask_blocks(const bsa_mask_desc* d) {
 
 extern "C" {
 
-int32_t bsa_version(void) { return 100; }
+int32_t bsa_version(void) { return 110; }
 
 const char* bsa_status_string(int32_t code) {
   switch (code) {
@@ -56,6 +57,7 @@ const char* bsa_status_string(int32_t code) {
     case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
     case BSA_ERR_CAPACITY: return "BSA_ERR_CAPACITY";
     case BSA_ERR_SCRATCH_LIMIT: return "BSA_ERR_SCRATCH_LIMIT";
+    case BSA_ERR_BAD_PADDING: return "BSA_ERR_BAD_PADDING";
     default: return "BSA_UNKNOWN_STATUS";
   }
 }
@@ -82,10 +84,10 @@ bsa_status bsa_build_mask(const bsa_mask_desc* desc, int32_t* row_ptr, int32_t* 
 }
 
 bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int32_t H, int32_t L,
-                          int32_t d, int32_t block, float* kbar, float* vsum, float* Hbar,
-                          float* Mnorm, float* Hblk, void* workspace, size_t ws_bytes,
-                          int32_t* status, void* stream) {
-  const Shape s{Bt, H, L, d, block};
+                          int32_t d, int32_t block, const int32_t* key_valid, float* kbar,
+                          float* vsum, float* Hbar, float* Mnorm, float* Hblk,
+                          void* workspace, size_t ws_bytes, int32_t* status, void* stream) {
+  const Shape s{Bt, H, L, d, block, key_valid};
   bsa_status r = check_shape(s);
   if (r != BSA_OK) return r;
   if (!K || !V || !kbar || !vsum || !Hbar || !Mnorm) return BSA_ERR_INVALID_ARG;
@@ -98,10 +100,10 @@ bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int32_t H, i
 }
 
 bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32_t Bt,
-                     int32_t H, int32_t L, int32_t d, int32_t block, int32_t k_top,
-                     float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
-                     float* scores, int32_t* status, void* stream) {
-  const Shape s{Bt, H, L, d, block};
+                     int32_t H, int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
+                     int32_t k_top, float lambda, float scale, int32_t* row_ptr,
+                     int32_t* col_idx, float* scores, int32_t* status, void* stream) {
+  const Shape s{Bt, H, L, d, block, key_valid};
   bsa_status r = check_shape(s);
   if (r != BSA_OK) return r;
   if (!Q || !kbar || !Mnorm || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
@@ -115,12 +117,13 @@ bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32
 }
 
 bsa_status bsa_forward(const void* Q, const void* K, const void* V, int32_t Bt, int32_t H,
-                       int32_t L, int32_t d, int32_t block, const int32_t* row_ptr,
+                       int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
+                       const int32_t* row_ptr,
                        const int32_t* col_idx, int64_t nnz_total, int32_t csr_per_head,
                        int32_t mode, const float* kbar, const float* vsum,
                        const float* Hbar, float scale, void* O, float* lse,
                        void* workspace, size_t ws_bytes, int32_t* status, void* stream) {
-  const Shape s{Bt, H, L, d, block};
+  const Shape s{Bt, H, L, d, block, key_valid};
   bsa_status r = check_shape(s);
   if (r != BSA_OK) return r;
   if (!Q || !K || !V || !O || !row_ptr) return BSA_ERR_INVALID_ARG;

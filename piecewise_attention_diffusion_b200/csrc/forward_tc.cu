@@ -79,6 +79,7 @@ struct Params {
   int csr_per_head;
   int pisa;
   int linear;  // per-block first order: every block a tile, unselected ones linearised
+  const int32_t* key_valid;  // real tokens per block, or null (no padding)
   float scale, scale_log2;
   __nv_bfloat16* O;
   float* lse;
@@ -595,13 +596,11 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             else if (valid < lo + 32) excl[w] |= 0xffffffffu << (valid - lo);
           }
         }
-        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
         bool skip = false;          // whole tile masked for this row
         bool lin = false;           // block t unselected for this row (per-block mode)
+        int jt = -1;                // key block of an exact tile (needed with padding)
         if (kLinear) {
+          jt = t;
           if (nxt == t) {
             ++mp;
             nxt = mp < me ? __ldg(p.col_idx + mp) : INT_MAX;
@@ -609,11 +608,31 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             lin = true;
           }
         } else if (!chunk && C::QBPT == 2) {
-          const int j = lists.next();
-          const bool member = mp < me && __ldg(p.col_idx + mp) == j;
+          jt = lists.next();
+          const bool member = mp < me && __ldg(p.col_idx + mp) == jt;
           if (member) ++mp;
           skip = !member;
+        } else if (!chunk && p.key_valid != nullptr) {
+          jt = __ldg(p.col_idx + mb + t);   // one query block per tile: its own list
         }
+        // token padding: an exact tile of a block with fewer real tokens than its width
+        // excludes its tail columns (the same exclusion bits as a centroid chunk)
+        bool masked = false;
+        if (!chunk && p.key_valid != nullptr && jt >= 0) {
+          const int v = min(max(__ldg(p.key_valid + jt), 1), BKV);
+          if (v < BKV) {
+            masked = true;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int lo = w * 32;
+              excl[w] = v <= lo ? 0xffffffffu : (v < lo + 32 ? 0xffffffffu << (v - lo) : 0u);
+            }
+          }
+        }
+        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
         // pass 1: this thread's whole S row into registers (one wait), the excluded
         // entries of a centroid chunk set to -inf, then the row max
         const int cols = chunk ? kChunk : BKV;
@@ -627,7 +646,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             tmem_ld32(s_base + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
           }
           tmem_wait_ld();
-          if (chunk) {
+          if (chunk || masked) {
 #pragma unroll
             for (int e = 0; e < 128; ++e)
               if ((excl[e >> 5] >> (e & 31)) & 1u) r[e] = __float_as_uint(-INFINITY);
@@ -678,6 +697,8 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           rs = (float)BKV * alpha;
         } else if (chunk) {
           rs = row_exp<128, false>(r, p.scale_log2, m_ref, s_base);
+        } else if (masked) {  // -inf entries: the special-function unit gives exact zeros
+          rs = row_exp<BKV, false>(r, p.scale_log2, m_ref, s_base);
         } else {
           rs = row_exp<BKV, true>(r, p.scale_log2, m_ref, s_base);
         }
@@ -865,6 +886,7 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.csr_per_head = a.csr_per_head;
   p.pisa = a.mode == BSA_MODE_PISA;
   p.linear = a.mode == BSA_MODE_PISA_BLOCK;
+  p.key_valid = s.key_valid;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.O = static_cast<__nv_bfloat16*>(a.O);

@@ -9,6 +9,7 @@ namespace bsa {
 
 struct Shape {
   int Bt, H, L, d, block;
+  const int32_t* key_valid = nullptr;  // real tokens per block (device int32 [M]), or null
   int BH() const { return Bt * H; }
   int M() const { return L / block; }
 };

@@ -53,17 +53,19 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 extern "C" bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void* V,
                                           int32_t Bt, int32_t H, int32_t L, int32_t d,
-                                          int32_t block, const int32_t* row_ptr,
+                                          int32_t block, const int32_t* key_valid,
+                                          const int32_t* row_ptr,
                                           const int32_t* col_idx, int64_t nnz_total,
                                           int32_t csr_per_head, int32_t mode, const float* kbar,
                                           const float* vsum, const float* Hbar, float scale,
                                           void* O, float* lse, int32_t* status, void* stream) {
-  const bsa::Shape s{Bt, H, L, d, block};
+  const bsa::Shape s{Bt, H, L, d, block, key_valid};
   if (Bt <= 0 || H <= 0 || L <= 0 || d <= 0 || block <= 0) return BSA_ERR_INVALID_ARG;
   if ((d != 64 && d != 128) || (block != 64 && block != 128) || L % block != 0 ||
       s.M() > 2048 || (int64_t)Bt * H > 65535 || (int64_t)Bt * H * L * d >= (int64_t)1 << 40)
     return BSA_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !O || !row_ptr) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(key_valid) & 3u) != 0) return BSA_ERR_INVALID_ARG;
   if (nnz_total < 0 || (nnz_total > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
   if (nnz_total >= INT32_MAX) return BSA_ERR_UNSUPPORTED;
   if (!bsa::aligned16(Q) || !bsa::aligned16(K) || !bsa::aligned16(V) || !bsa::aligned16(O))

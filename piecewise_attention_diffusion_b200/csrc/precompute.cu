@@ -125,10 +125,33 @@ __device__ __forceinline__ void for_each_acc(float (&acc)[Tiling<D>::MT][Tiling<
       }
 }
 
-// Column means of K and column sums of V of the resident tile (threads 0..2D-1).
+// Token padding: the block's rows past its nv real tokens are zeroed in both resident
+// tiles, so that the column sums and K^T V below run over the real tokens only.
+template <int B, int D>
+__device__ __forceinline__ void zero_padding(__nv_bfloat16* Ks, __nv_bfloat16* Vs, int nv) {
+  constexpr int P = TilePitch<D>::elems;
+  for (int e = threadIdx.x; e < (B - nv) * D; e += kThreads) {
+    const int r = nv + e / D, c = e % D;
+    Ks[r * P + c] = __float2bfloat16(0.f);
+    Vs[r * P + c] = __float2bfloat16(0.f);
+  }
+}
+
+// Real tokens of block j (B without padding); an out-of-range count is reported and
+// clamped.
+template <int B>
+__device__ __forceinline__ int real_tokens(const int32_t* key_valid, int j, int32_t* status) {
+  if (key_valid == nullptr) return B;
+  const int raw = __ldg(key_valid + j);
+  if ((raw < 1 || raw > B) && threadIdx.x == 0) report(status, BSA_ERR_BAD_PADDING);
+  return min(max(raw, 1), B);
+}
+
+// Column means of K and column sums of V of the resident tile (threads 0..2D-1), over
+// the block's nv real tokens (the padded rows are zero).
 template <int B, int D>
 __device__ __forceinline__ void column_stats(const __nv_bfloat16* Ks, const __nv_bfloat16* Vs,
-                                             float* s_kbar, float* s_vsum) {
+                                             float* s_kbar, float* s_vsum, int nv) {
   constexpr int P = TilePitch<D>::elems;
   const int t = threadIdx.x;
   if (t < 2 * D) {
@@ -139,7 +162,7 @@ __device__ __forceinline__ void column_stats(const __nv_bfloat16* Ks, const __nv
 #pragma unroll 8
     for (int n = 0; n < B; ++n) s += __bfloat162float(src[n * P + c]);
     if (is_k)
-      s_kbar[c] = s * (1.0f / B);
+      s_kbar[c] = s / (float)nv;
     else
       s_vsum[c] = s;
   }
@@ -148,8 +171,8 @@ __device__ __forceinline__ void column_stats(const __nv_bfloat16* Ks, const __nv
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
 k_pre_stats(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int L,
-            int G, float* __restrict__ kbar, float* __restrict__ vsum,
-            float* __restrict__ partial) {
+            int G, const int32_t* __restrict__ key_valid, float* __restrict__ kbar,
+            float* __restrict__ vsum, float* __restrict__ partial, int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int P = TilePitch<D>::elems;
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem);
@@ -168,7 +191,12 @@ k_pre_stats(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict
     load_tile_async<B, D>(Vs, V + head + (size_t)j * B * D);
     cp_async_wait_all();
     __syncthreads();
-    column_stats<B, D>(Ks, Vs, s_kbar, s_vsum);
+    const int nv = real_tokens<B>(key_valid, j, status);
+    if (nv < B) {
+      zero_padding<B, D>(Ks, Vs, nv);
+      __syncthreads();
+    }
+    column_stats<B, D>(Ks, Vs, s_kbar, s_vsum, nv);
     ktv_accumulate<B, D>(acc, Ks, Vs);
     __syncthreads();
     if (threadIdx.x < D) {
@@ -198,7 +226,8 @@ __global__ void k_pre_reduce(const float* __restrict__ partial, int n_grp, int D
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
 k_pre_norm(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int L,
-           const float* __restrict__ Hbar, float* __restrict__ Mnorm, float* __restrict__ Hblk) {
+           const int32_t* __restrict__ key_valid, const float* __restrict__ Hbar,
+           float* __restrict__ Mnorm, float* __restrict__ Hblk, int32_t* status) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int P = TilePitch<D>::elems;
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(smem);
@@ -214,7 +243,12 @@ k_pre_norm(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
   load_tile_async<B, D>(Vs, V + head + (size_t)j * B * D);
   cp_async_wait_all();
   __syncthreads();
-  column_stats<B, D>(Ks, Vs, s_kbar, s_vsum);
+  const int nv = real_tokens<B>(key_valid, j, status);
+  if (nv < B) {
+    zero_padding<B, D>(Ks, Vs, nv);
+    __syncthreads();
+  }
+  column_stats<B, D>(Ks, Vs, s_kbar, s_vsum, nv);
   float acc[Tiling<D>::MT][Tiling<D>::NT][4] = {};
   ktv_accumulate<B, D>(acc, Ks, Vs);
   __syncthreads();
@@ -253,7 +287,8 @@ size_t smem_bytes() {
 
 template <int B, int D>
 cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float* vsum,
-                float* Hbar, float* Mnorm, float* Hblk, void* ws, cudaStream_t st) {
+                float* Hbar, float* Mnorm, float* Hblk, void* ws, int32_t* status,
+                cudaStream_t st) {
   const int M = s.M(), G = group_size(s), n_grp = ceil_div(M, G);
   const size_t sm = smem_bytes<B, D>();
   cudaError_t e;
@@ -266,13 +301,14 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   float* partial = static_cast<float*>(ws);
   const auto* Kb = static_cast<const __nv_bfloat16*>(K);
   const auto* Vb = static_cast<const __nv_bfloat16*>(V);
-  k_pre_stats<B, D><<<dim3(n_grp, s.BH()), kThreads, sm, st>>>(Kb, Vb, s.L, G, kbar, vsum,
-                                                               partial);
+  k_pre_stats<B, D><<<dim3(n_grp, s.BH()), kThreads, sm, st>>>(Kb, Vb, s.L, G, s.key_valid,
+                                                               kbar, vsum, partial, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   k_pre_reduce<<<dim3(ceil_div(D * D, 256), s.BH()), 256, 0, st>>>(partial, n_grp, D * D, M,
                                                                    Hbar);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_pre_norm<B, D><<<dim3(M, s.BH()), kThreads, sm, st>>>(Kb, Vb, s.L, Hbar, Mnorm, Hblk);
+  k_pre_norm<B, D><<<dim3(M, s.BH()), kThreads, sm, st>>>(Kb, Vb, s.L, s.key_valid, Hbar,
+                                                          Mnorm, Hblk, status);
   return cudaGetLastError();
 }
 
@@ -291,8 +327,8 @@ cudaError_t launch_precompute(const Shape& s, const void* K, const void* V, floa
   // different TMEM layout) keeps the mma.sync kernels of this file
   if (s.d == 128)
     return launch_precompute_tc(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
-  if (s.block == 64) return run<64, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
-  return run<128, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, st);
+  if (s.block == 64) return run<64, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+  return run<128, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
 }
 
 }  // namespace bsa

@@ -57,6 +57,7 @@ struct Params {
   const float* Hbar;      // norm
   float* Mnorm;           // norm
   float* Hblk;            // norm, nullable
+  const int32_t* key_valid;  // real tokens per block, or null (no padding)
   int32_t* status;
 };
 
@@ -166,21 +167,42 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_c = idesc_bf16_f32(128, D, true, true);
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, true, false);
-      const uint32_t ones = smem_u32(sOnes);
-      BlockIter it;
-      it.init(p);
-      uint32_t n = 0;
-      bool ok = true;
-      while (it.valid()) {
-        const int st = n % kStages, b = n & 1;
-        ok = mbar_wait(&bars.full[st], (n / kStages) & 1, abort_flag);
-        if (ok && n >= 2) ok = mbar_wait(&bars.tmem_free[b], ((n >> 1) - 1) & 1, abort_flag);
-        if (!ok) break;
+    // Lane 0 issues; with token padding the whole warp first zeroes the tail rows of a
+    // padded block's K and V tiles, so that every product and column sum runs over the
+    // real tokens only (a row fills 128 bytes of each 64-column sub-tile, whatever the
+    // swizzle).
+    constexpr uint32_t idesc_c = idesc_bf16_f32(128, D, true, true);
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, true, false);
+    const uint32_t ones = smem_u32(sOnes);
+    BlockIter it;
+    it.init(p);
+    uint32_t n = 0;
+    bool ok = true;
+    while (it.valid()) {
+      const int st = n % kStages, b = n & 1;
+      ok = mbar_wait(&bars.full[st], (n / kStages) & 1, abort_flag);
+      if (ok && n >= 2) ok = mbar_wait(&bars.tmem_free[b], ((n >> 1) - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      unsigned char* stage = smem + st * C::STAGE;
+      if (p.key_valid != nullptr) {
+        const int v = min(max(__ldg(p.key_valid + it.j), 1), B);
+        if (v < B) {
+          constexpr int kChunks = (D / 64) * 8;  // 16-byte chunks of one row
+          for (int e = lane; e < 2 * (B - v) * kChunks; e += 32) {
+            const int tile = e / ((B - v) * kChunks), rest = e % ((B - v) * kChunks);
+            const int r = v + rest / kChunks, c = rest % kChunks;
+            *reinterpret_cast<uint4*>(stage + tile * C::TILE + (c / 8) * (B * 128) + r * 128 +
+                                      (c % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          // the tensor core (async proxy) reads what these generic stores wrote
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+      }
+      if (lane == 0) {
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + st * C::STAGE);
+        const uint32_t k_addr = smem_u32(stage);
         const uint32_t v_addr = k_addr + C::TILE;
         const uint32_t dc = tmem + 256u * b;
 #pragma unroll
@@ -194,9 +216,12 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         }
         mma_commit(&bars.empty[st]);
         mma_commit(&bars.mma_done[b]);
-        ++n;
-        it.next();
       }
+      __syncwarp();
+      ++n;
+      it.next();
+    }
+    if (lane == 0) {
       mma_commit(&bars.done);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(&bars.done, 0) && globaltimer_ns() - t0 < 100000000ull) {
@@ -244,7 +269,13 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         tmem_ld16(base + 128, r0);
         tmem_ld16(base + 144, r1);
         tmem_wait_ld();
-        kb = __uint_as_float(r0[0]) * (1.0f / B);
+        int nv = B;  // real tokens of the block
+        if (p.key_valid != nullptr) {
+          const int raw = __ldg(p.key_valid + j);
+          if ((raw < 1 || raw > B) && a == 0) report(p.status, BSA_ERR_BAD_PADDING);
+          nv = min(max(raw, 1), B);
+        }
+        kb = __uint_as_float(r0[0]) / (float)nv;
         vs = __uint_as_float(r1[0]);
       }
       if (kStats) {
@@ -405,6 +436,7 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   p.Hbar = Hbar;
   p.Mnorm = Mnorm;
   p.Hblk = Hblk;
+  p.key_valid = s.key_valid;
   p.status = status;
   // both passes deal the flattened (head, block) range in contiguous pieces, one per CTA
   p.n_units = s.BH() * M;

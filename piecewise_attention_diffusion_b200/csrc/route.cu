@@ -19,6 +19,11 @@
 //      patterns (scores are >= 0, so the bit patterns order like the values), ties at
 //      the threshold go to the smaller block index, and the selected indices are
 //      compacted in ascending order with ordered ballots.
+// Token padding: the pooled query of a block averages its real rows only, and every
+// padded block (fewer than B real tokens) is forced into every list. It takes the key
+// +inf in the selection (scores are finite), so the radix select, the tie rule and the
+// compaction treat it as the largest score without a separate pass; the scores
+// written out keep the real values.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,13 +32,14 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
+constexpr uint32_t kForcedKey = 0x7F800000u;  // bit pattern of +inf
 
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
 k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
-        const float* __restrict__ Mnorm, int L, int k_top, float lambda, float scale,
-        int32_t* __restrict__ row_ptr, int32_t* __restrict__ col_idx,
-        float* __restrict__ scores) {
+        const float* __restrict__ Mnorm, const int32_t* __restrict__ key_valid, int L,
+        int k_top, float lambda, float scale, int32_t* __restrict__ row_ptr,
+        int32_t* __restrict__ col_idx, float* __restrict__ scores, int32_t* status) {
   const int M = L / B;
   const int bh = blockIdx.y;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -67,14 +73,22 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   if (active) {
     const __nv_bfloat16* qb = Q + ((size_t)bh * L + (size_t)i * B) * D;
     const int cc = lane % CPR, r0 = lane / CPR;
+    int nq = B;  // real query rows of block i
+    if (key_valid != nullptr) {
+      const int raw = __ldg(key_valid + i);
+      if ((raw < 1 || raw > B) && lane == 0) report(status, BSA_ERR_BAD_PADDING);
+      nq = min(max(raw, 1), B);
+    }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll kUnrollQ
     for (int r = r0; r < B; r += RPI) {
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(qb + (size_t)r * D) + cc);
       float f[8];
       bf16x8_to_f32(u, f);
+      if (r < nq) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+      }
     }
 #pragma unroll
     for (int o = CPR; o < 32; o <<= 1)
@@ -82,7 +96,7 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
       for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
     if (lane < CPR) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qbar[cc * 8 + e] = acc[e] * (1.0f / B);
+      for (int e = 0; e < 8; ++e) qbar[cc * 8 + e] = acc[e] / (float)nq;
     }
   }
   __syncwarp();
@@ -133,10 +147,20 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   se = warp_sum(se);
   const float inv_se = 1.0f / se;
   float* srow = scores ? scores + ((size_t)bh * M + i) * M : nullptr;
+  int n_forced = 0;
   for (int j = lane; j < M; j += 32) {
     const float v = expf(sc[j] - mx) * inv_se + s_cov[j];
-    sc[j] = v;
+    const bool forced = key_valid != nullptr && __ldg(key_valid + j) < B;
+    n_forced += forced ? 1 : 0;
+    sc[j] = forced ? __uint_as_float(kForcedKey) : v;
     if (srow) srow[j] = v;
+  }
+  n_forced = __reduce_add_sync(0xffffffffu, n_forced);
+  if (n_forced > k_top) {
+    // the list cannot hold every padded block: report, and emit a valid list anyway
+    if (lane == 0) report(status, BSA_ERR_BAD_PADDING);
+    for (int j = lane; j < M; j += 32)
+      if (__float_as_uint(sc[j]) == kForcedKey) sc[j] = 0.f;
   }
   __syncwarp();
 
@@ -180,15 +204,15 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
 template <int B, int D>
 cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* Mnorm,
                 int k_top, float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
-                float* scores, cudaStream_t st) {
+                float* scores, int32_t* status, cudaStream_t st) {
   const int M = s.M();
   const size_t sm = ((size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(k_route<B, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   k_route<B, D><<<dim3(ceil_div(M, kWarps), s.BH()), kThreads, sm, st>>>(
-      static_cast<const __nv_bfloat16*>(Q), kbar, Mnorm, s.L, k_top, lambda, scale, row_ptr,
-      col_idx, scores);
+      static_cast<const __nv_bfloat16*>(Q), kbar, Mnorm, s.key_valid, s.L, k_top, lambda, scale,
+      row_ptr, col_idx, scores, status);
   return cudaGetLastError();
 }
 
@@ -197,14 +221,17 @@ cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* M
 cudaError_t launch_route(const Shape& s, const void* Q, const float* kbar, const float* Mnorm,
                          int k_top, float lambda, float scale, int32_t* row_ptr,
                          int32_t* col_idx, float* scores, int32_t* status, cudaStream_t st) {
-  (void)status;
   if (s.block == 64 && s.d == 64)
-    return run<64, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, st);
+    return run<64, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
+                        status, st);
   if (s.block == 64 && s.d == 128)
-    return run<64, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, st);
+    return run<64, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
+                         status, st);
   if (s.block == 128 && s.d == 64)
-    return run<128, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, st);
-  return run<128, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, st);
+    return run<128, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
+                         status, st);
+  return run<128, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
+                          status, st);
 }
 
 }  // namespace bsa

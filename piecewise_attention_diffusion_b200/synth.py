@@ -11,12 +11,21 @@ values the GPU sees upcast the bf16 tensors.
 Workloads (sizes named after what they are):
   * tiny_pisa          batch 1, 2 heads, L=512, d=64, block 64
   * multimodal_dit     batch 8, 16 heads, L=1152 (77 text tokens padded to 128 +
-                       32x32 image patches), d=64, block 64
-  * multimodal_pisa    the same shape and fixed mask as the exact set of PISA
+                       32x32 image patches), d=64, block 64; the 51 pad tokens are
+                       marked (real tokens per block 64, 13, 64, ...)
+  * multimodal_pisa    the same shape, padding and fixed mask as the exact set of PISA
+  * text_image_pisa    batch 1, 24 heads, L=4352: 77 text tokens padded to a 128-block,
+                       a 64x64 latent (32 blocks), a timestep token padded to a
+                       128-block; d=128, block 128, routed PISA at 15% density
   * image_pisa_block, video_pisa_block   the per-block first-order form of PISA
   * image_pisa         batch 1, 24 heads, L=4096 (64x64 latent), d=128, block 128
   * video_pisa         batch 1, 40 heads, L=16384 (16 frames x 32x32), d=128, block 128
   * sweep_L{L}         batch 1, 24 heads, L in {4096..32768}, d=128, block 128
+
+Token padding: a workload with ``key_valid`` marks the leading real tokens of each
+block; the pad rows of k and v are filled with large noise (4 x N(0,1)) and those of q
+with N(0,1), from a generator of their own, so that any leak of a pad key into a result
+shows, and the real rows are the same draws as in the unpadded workload.
 """
 from __future__ import annotations
 
@@ -41,10 +50,15 @@ class Workload:
     generator: str = "iid"        # iid | block_centres | field2d_hot | field3d
     grid: tuple = ()              # spatial token grid for the field generators
     mask: dict = field(default_factory=dict)  # fixed multimodal mask descriptor
+    key_valid: tuple = ()         # real tokens per block (empty: no padding)
 
     @property
     def n_blocks(self) -> int:
         return self.seq_len // self.block
+
+    def valid_tokens(self) -> list | None:
+        """Real tokens per block as a list of M ints, or None without padding."""
+        return list(self.key_valid) if self.key_valid else None
 
     def top_k(self) -> int:
         """Blocks per query block computed exactly: k = max(1, ceil(density*M))."""
@@ -63,11 +77,16 @@ def workloads() -> dict:
     w["multimodal_dit"] = Workload(
         "multimodal_dit", 8, 16, 1152, 64, 64, "keep_or_drop", generator="iid",
         mask=dict(n_text_blocks=2, grid_h=4, grid_w=4, radius=1, global_stride=16,
-                  global_rows_full=0))
+                  global_rows_full=0),
+        key_valid=(64, 13) + (64,) * 16)
     # the same fixed pattern as the selection of PISA: the blocks it drops enter through
     # the Taylor tail (zeroth order per block, first order through Hbar)
     w["multimodal_pisa"] = dataclasses.replace(w["multimodal_dit"], name="multimodal_pisa",
                                                mode="pisa")
+    # text block (77 of 128 real), 32 latent blocks, timestep block (1 of 128 real)
+    w["text_image_pisa"] = Workload("text_image_pisa", 1, 24, 4352, 128, 128, "pisa",
+                                    density=0.15, generator="block_centres",
+                                    key_valid=(77,) + (128,) * 32 + (1,))
     w["image_pisa"] = Workload("image_pisa", 1, 24, 4096, 128, 128, "pisa", density=0.15,
                                generator="field2d_hot", grid=(64, 64))
     w["video_pisa"] = Workload("video_pisa", 1, 40, 16384, 128, 128, "pisa", density=0.125,
@@ -143,6 +162,12 @@ def make_qkv(w: Workload, seed: int = 0, heads: list | None = None) -> tuple:
             v = _smooth_field(g, w.grid, d) + 0.3 * torch.randn(L, d, generator=g)
         else:
             raise ValueError(f"unknown generator {w.generator}")
+        if w.key_valid:
+            gp = torch.Generator().manual_seed(seed * 1_000_003 + bh * 7919 + 29)
+            for j, n in enumerate(w.key_valid):
+                if n < B:
+                    for x, amp in ((q, 1.0), (k, 4.0), (v, 4.0)):
+                        x[j * B + n:(j + 1) * B] = amp * torch.randn(B - n, d, generator=gp)
         qs.append(q)
         ks.append(k)
         vs.append(v)

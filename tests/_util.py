@@ -33,13 +33,19 @@ def assert_close_out(got, want, what=""):
     return mx, rl
 
 
-def rows_agree_up_to_ties(gpu_cols, orc_cols, orc_scores_row, k_top):
+def rows_agree_up_to_ties(gpu_cols, orc_cols, orc_scores_row, k_top, forced=()):
     """True if the selected sets are equal, or differ only in blocks whose oracle score
-    is within TIE_REL_TOL (relative) of the oracle's k-th largest score."""
+    is within TIE_REL_TOL (relative) of the oracle's k-th largest score. ``forced``
+    blocks (padded ones) must be in both sets; the threshold is then the
+    (k_top - len(forced))-th largest score among the other blocks."""
     g, o = set(int(x) for x in gpu_cols), set(int(x) for x in orc_cols)
+    fset = set(int(x) for x in forced)
+    if not (fset <= g and fset <= o):
+        return False
     if g == o:
         return True
     s = np.asarray(orc_scores_row, dtype=np.float64)
-    kth = np.sort(s)[::-1][k_top - 1]
+    free = np.asarray([s[j] for j in range(len(s)) if j not in fset])
+    kth = np.sort(free)[::-1][k_top - len(fset) - 1]
     tol = TIE_REL_TOL * max(abs(kth), 1e-30)
     return all(abs(s[j] - kth) <= tol for j in g ^ o)

@@ -67,7 +67,7 @@ def _fake(n=1 << 20):
     (64, 64, 64 * 4096, b.ERR_UNSUPPORTED)])
 def test_forward_rejects_unsupported_shapes(d, block, L, want):
     p = _fake()
-    rc = b.lib().bsa_forward(p, p, p, 1, 2, L, d, block, p, p, 8, 0, 0, None, None, None,
+    rc = b.lib().bsa_forward(p, p, p, 1, 2, L, d, block, None, p, p, 8, 0, 0, None, None, None,
                              0.0, p, None, p, 1 << 20, None, None)
     assert rc == want
 
@@ -78,40 +78,45 @@ def test_forward_rejects_bad_arguments():
     f = b.lib().bsa_forward
     common = (1, 2, 256, 64, 64)
     # misaligned Q
-    assert f(mis, p, p, *common, p, p, 8, 0, 0, None, None, None, 0.0, p, None, p, 1 << 20,
+    assert f(mis, p, p, *common, None, p, p, 8, 0, 0, None, None, None, 0.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
     # PISA without statistics
-    assert f(p, p, p, *common, p, p, 8, 0, 1, None, None, None, 0.0, p, None, p, 1 << 20,
+    assert f(p, p, p, *common, None, p, p, 8, 0, 1, None, None, None, 0.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
     # bad mode / csr flag / negative scale / negative nnz
-    assert f(p, p, p, *common, p, p, 8, 0, 7, None, None, None, 0.0, p, None, p, 1 << 20,
+    assert f(p, p, p, *common, None, p, p, 8, 0, 7, None, None, None, 0.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
-    assert f(p, p, p, *common, p, p, 8, 3, 0, None, None, None, 0.0, p, None, p, 1 << 20,
+    assert f(p, p, p, *common, None, p, p, 8, 3, 0, None, None, None, 0.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
-    assert f(p, p, p, *common, p, p, 8, 0, 0, None, None, None, -1.0, p, None, p, 1 << 20,
+    assert f(p, p, p, *common, None, p, p, 8, 0, 0, None, None, None, -1.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
-    assert f(p, p, p, *common, p, p, -1, 0, 0, None, None, None, 0.0, p, None, p, 1 << 20,
+    assert f(p, p, p, *common, None, p, p, -1, 0, 0, None, None, None, 0.0, p, None, p, 1 << 20,
              None, None) == b.ERR_INVALID_ARG
     # missing / short workspace
-    assert f(p, p, p, *common, p, p, 8, 0, 0, None, None, None, 0.0, p, None, None, 0,
+    assert f(p, p, p, *common, None, p, p, 8, 0, 0, None, None, None, 0.0, p, None, None, 0,
              None, None) == b.ERR_WORKSPACE
-    assert f(p, p, p, *common, p, p, 8, 0, 0, None, None, None, 0.0, p, None, p, 8,
+    assert f(p, p, p, *common, None, p, p, 8, 0, 0, None, None, None, 0.0, p, None, p, 8,
              None, None) == b.ERR_WORKSPACE
 
 
 def test_route_and_precompute_reject_bad_arguments():
     p = _fake()
     r = b.lib().bsa_route
-    assert r(p, p, p, 1, 2, 512, 64, 64, 0, 1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 0, 1.0, 0.0, p, p, None, None, None) == \
         b.ERR_INVALID_ARG                                      # k_top 0
-    assert r(p, p, p, 1, 2, 512, 64, 64, 9, 1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 9, 1.0, 0.0, p, p, None, None, None) == \
         b.ERR_INVALID_ARG                                      # k_top > M
-    assert r(p, p, p, 1, 2, 512, 64, 64, 2, -1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 2, -1.0, 0.0, p, p, None, None, None) == \
         b.ERR_INVALID_ARG                                      # lambda < 0
+    odd = ctypes.c_void_p((1 << 20) + 2)                       # key_valid not 4-aligned
+    assert r(p, p, p, 1, 2, 512, 64, 64, odd, 2, 1.0, 0.0, p, p, None, None, None) == \
+        b.ERR_INVALID_ARG
     pc = b.lib().bsa_precompute
-    assert pc(p, p, 1, 2, 512, 64, 64, p, p, p, p, None, None, 0, None, None) == \
+    assert pc(p, p, 1, 2, 512, 64, 64, None, p, p, p, p, None, None, 0, None, None) == \
         b.ERR_WORKSPACE
-    assert pc(p, None, 1, 2, 512, 64, 64, p, p, p, p, None, p, 1 << 30, None, None) == \
+    assert pc(p, None, 1, 2, 512, 64, 64, None, p, p, p, p, None, p, 1 << 30, None, None) == \
+        b.ERR_INVALID_ARG
+    assert pc(p, p, 1, 2, 512, 64, 64, odd, p, p, p, p, None, p, 1 << 30, None, None) == \
         b.ERR_INVALID_ARG
 
 

@@ -132,16 +132,18 @@ def test_route_parity_on_oracle_statistics(name, heads, lam):
 
 # ------------------------------------------------------------------------- forward
 def _forward_check(w, q, k, v, rp, ci, per_head, mode, stats_np, qblocks=None, heads_idx=None,
-                   lse_check=True):
-    """Run bsa_forward on all heads; compare the requested heads / query blocks."""
+                   lse_check=True, key_valid=None):
+    """Run bsa_forward on all heads; compare the requested heads / query blocks.
+    ``key_valid`` (real tokens per block) goes to both sides."""
     BH = q.shape[0] * q.shape[1]
     M = w.seq_len // w.block
     scale = 1 / math.sqrt(w.head_dim)
     grp, gci = _csr_to_gpu(rp, ci)
     st = _status()
     stats = _stats_to_gpu(*stats_np[:3]) if mode == b.MODE_PISA else None
+    kv = None if key_valid is None else torch.tensor(key_valid, dtype=torch.int32, device=DEV)
     O, lse = b.forward(q.to(DEV), k.to(DEV), v.to(DEV), w.block, grp, gci, per_head, mode,
-                       stats=stats, want_lse=True, status=st)
+                       stats=stats, want_lse=True, status=st, key_valid=kv)
     torch.cuda.synchronize()
     assert st.item() == 0
     Og = O.reshape(BH, w.seq_len, w.head_dim)
@@ -154,14 +156,15 @@ def _forward_check(w, q, k, v, rp, ci, per_head, mode, stats_np, qblocks=None, h
         if mode == b.MODE_PISA:
             kbar, vsum, Hbar = (x[h] for x in stats_np[:3])
             want, wl = orc.pisa_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale, kbar,
-                                     vsum, Hbar, qblocks=blocks)
+                                     vsum, Hbar, qblocks=blocks, key_valid=key_valid)
         elif mode == b.MODE_PISA_BLOCK:
             kbar, vsum, Hbar, Hblk = (x[h] for x in stats_np)
             want, wl = orc.pisa_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale, kbar,
-                                     vsum, Hbar, qblocks=blocks, Hblocks=Hblk)
+                                     vsum, Hbar, qblocks=blocks, Hblocks=Hblk,
+                                     key_valid=key_valid)
         else:
             want, wl = orc.keep_or_drop_head(qf[h], kf[h], vf[h], hrp, hci, w.block, scale,
-                                             qblocks=blocks)
+                                             qblocks=blocks, key_valid=key_valid)
         rows = np.concatenate([np.arange(i * w.block, (i + 1) * w.block) for i in blocks])
         mx, rl = assert_close_out(Og[h, rows], want, f"head {h}")
         worst = (max(worst[0], mx), max(worst[1], rl))
@@ -200,12 +203,14 @@ def test_forward_tiny_random_lists(mode):
 
 
 def test_forward_multimodal_fixed_mask_keep_or_drop():
+    """77 text tokens in two 64-blocks (13 real in the second): the 51 pad keys, filled
+    with large noise, must not reach any output row."""
     w = synth.workloads()["multimodal_dit"]
     q, k, v = synth.make_qkv(w)
     keep = orc.mask_dense(**w.mask)
     rp, ci = orc.dense_to_csr(keep)
     _forward_check(w, q, k, v, rp, ci, 0, b.MODE_KEEP_OR_DROP, None,
-                   heads_idx=[0, 17, 63, 127])
+                   heads_idx=[0, 17, 63, 127], key_valid=w.valid_tokens())
 
 
 def test_forward_pisa_over_the_multimodal_fixed_mask():
@@ -220,11 +225,12 @@ def test_forward_pisa_over_the_multimodal_fixed_mask():
     BH = w.batch * w.heads
     kf = f64(k).reshape(BH, w.seq_len, w.head_dim)
     vf = f64(v).reshape(BH, w.seq_len, w.head_dim)
-    stats = [orc.precompute_head(kf[h], vf[h], w.block) for h in range(BH)]
+    stats = [orc.precompute_head(kf[h], vf[h], w.block, w.valid_tokens()) for h in range(BH)]
     kbar = np.stack([s_[0] for s_ in stats])
     vsum = np.stack([s_[1] for s_ in stats])
     Hbar = np.stack([s_[3] for s_ in stats])
-    _forward_check(w, q, k, v, rp, ci, 0, b.MODE_PISA, (kbar, vsum, Hbar), heads_idx=heads)
+    _forward_check(w, q, k, v, rp, ci, 0, b.MODE_PISA, (kbar, vsum, Hbar), heads_idx=heads,
+                   key_valid=w.valid_tokens())
 
 
 @pytest.mark.parametrize("L,block,d,kk", [(576, 64, 64, 3), (640, 128, 128, 2), (64, 64, 128, 1),
@@ -372,6 +378,7 @@ def test_forward_malformed_lists_set_status_and_leave_output():
     ("image_pisa", [0, 13], None),
     ("video_pisa", [0, 39], [0, 1, 63, 127]),
     ("sweep_L32768_d125_pisa", [0, 23], [0, 100, 255]),
+    ("text_image_pisa", [0, 11, 23], None),
 ])
 def test_pipeline_full_size_sampled(name, heads, qblocks):
     _pipeline_sampled(synth.workloads()[name], heads, qblocks)
@@ -391,14 +398,19 @@ def _pipeline_sampled(w, heads, qblocks):
 
     The forward for the sampled heads is run on the oracle's own block lists (spliced
     into the GPU-routed lists), so the output comparison does not depend on near-tie
-    routing decisions; the routing itself is compared separately with the tie rule."""
+    routing decisions; the routing itself is compared separately with the tie rule.
+    A workload with token padding passes its real-token counts to every call."""
     q, k, v = synth.make_qkv(w)
     kk, M, BH = w.top_k(), w.n_blocks, w.batch * w.heads
     scale = 1 / math.sqrt(w.head_dim)
     qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    valid = w.valid_tokens()
+    kv = None if valid is None else torch.tensor(valid, dtype=torch.int32, device=DEV)
+    forced = [] if valid is None else [j for j in range(M) if valid[j] < w.block]
     st = _status()
-    stats = b.precompute(kd, vd, w.block, status=st)
-    rp, ci, _ = b.route(qd, stats["kbar"], stats["Mnorm"], w.block, kk, 1.0, status=st)
+    stats = b.precompute(kd, vd, w.block, status=st, key_valid=kv)
+    rp, ci, _ = b.route(qd, stats["kbar"], stats["Mnorm"], w.block, kk, 1.0, status=st,
+                        key_valid=kv)
     torch.cuda.synchronize()
     assert st.item() == 0
     ci_host = ci.cpu().numpy().copy()
@@ -406,18 +418,19 @@ def _pipeline_sampled(w, heads, qblocks):
     for h in heads:
         bi, hh = divmod(h, w.heads)
         qf, kf, vf = f64(q[bi, hh]), f64(k[bi, hh]), f64(v[bi, hh])
-        kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block)
+        kbar, vsum, H, Hbar, Mn = orc.precompute_head(kf, vf, w.block, valid)
         np.testing.assert_allclose(f64(stats["Hbar"][h]), Hbar, atol=1e-3 * np.abs(Hbar).max())
-        orp, oci, osc = orc.route_head(qf, kbar, Mn, w.block, kk, 1.0, scale)
+        orp, oci, osc = orc.route_head(qf, kbar, Mn, w.block, kk, 1.0, scale, valid)
         g = ci_host[h * M * kk:(h + 1) * M * kk].reshape(M, kk)
         for i in range(M):
-            assert rows_agree_up_to_ties(g[i], oci[i * kk:(i + 1) * kk], osc[i], kk), (h, i)
+            assert rows_agree_up_to_ties(g[i], oci[i * kk:(i + 1) * kk], osc[i], kk,
+                                         forced), (h, i)
         ci_host[h * M * kk:(h + 1) * M * kk] = oci
         ref[h] = orc.pisa_head(qf, kf, vf, orp, oci, w.block, scale, kbar, vsum, Hbar,
-                               qblocks=qblocks)
+                               qblocks=qblocks, key_valid=valid)
     gci = torch.from_numpy(ci_host).to(DEV)
     O, lse = b.forward(qd, kd, vd, w.block, rp, gci, 1, b.MODE_PISA, stats=stats,
-                       want_lse=True, status=st)
+                       want_lse=True, status=st, key_valid=kv)
     torch.cuda.synchronize()
     assert st.item() == 0
     Og = O.reshape(BH, w.seq_len, w.head_dim)

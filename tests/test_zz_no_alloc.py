@@ -80,7 +80,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch(cuda_ok):
     # PISA on 256 heads of L = 32768, d = 128 needs about 40 MB > 16 MiB. Refused on the
     # host before any pointer is used or any kernel launched.
     p = ctypes.c_void_p(1 << 20)
-    rc = b.lib().bsa_forward_noalloc(p, p, p, 1, 256, 32768, 128, 128, p, p, 16, 1,
+    rc = b.lib().bsa_forward_noalloc(p, p, p, 1, 256, 32768, 128, 128, None, p, p, 16, 1,
                                      b.MODE_PISA, p, p, p, 0.0, p, None, None, None)
     assert rc == b.ERR_SCRATCH_LIMIT
     assert b.status_string(rc) == "BSA_ERR_SCRATCH_LIMIT"
