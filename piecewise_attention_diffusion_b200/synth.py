@@ -11,9 +11,11 @@ values the GPU sees upcast the bf16 tensors.
 Workloads (sizes named after what they are):
   * tiny_pisa          batch 1, 2 heads, L=512, d=64, block 64
   * multimodal_dit     batch 8, 16 heads, L=1152 (77 text tokens padded to 128 +
-                       32x32 image patches), d=64, block 64; the 51 pad tokens are
+                       32x32 image patches), d=64, block 64; every position is a
+                       real N(0,1) token (no token mask)
+  * multimodal_pisa    the same shape and fixed mask as the exact set of PISA
+  * multimodal_dit_padded, multimodal_pisa_padded   the same with the 51 pad tokens
                        marked (real tokens per block 64, 13, 64, ...)
-  * multimodal_pisa    the same shape, padding and fixed mask as the exact set of PISA
   * text_image_pisa    batch 1, 24 heads, L=4352: 77 text tokens padded to a 128-block,
                        a 64x64 latent (32 blocks), a timestep token padded to a
                        128-block; d=128, block 128, routed PISA at 15% density
@@ -77,12 +79,15 @@ def workloads() -> dict:
     w["multimodal_dit"] = Workload(
         "multimodal_dit", 8, 16, 1152, 64, 64, "keep_or_drop", generator="iid",
         mask=dict(n_text_blocks=2, grid_h=4, grid_w=4, radius=1, global_stride=16,
-                  global_rows_full=0),
-        key_valid=(64, 13) + (64,) * 16)
+                  global_rows_full=0))
     # the same fixed pattern as the selection of PISA: the blocks it drops enter through
     # the Taylor tail (zeroth order per block, first order through Hbar)
     w["multimodal_pisa"] = dataclasses.replace(w["multimodal_dit"], name="multimodal_pisa",
                                                mode="pisa")
+    # 77 text tokens: block 0 full, block 1 with 13 real tokens and 51 pad tokens
+    for n in ("multimodal_dit", "multimodal_pisa"):
+        w[n + "_padded"] = dataclasses.replace(w[n], name=n + "_padded",
+                                               key_valid=(64, 13) + (64,) * 16)
     # text block (77 of 128 real), 32 latent blocks, timestep block (1 of 128 real)
     w["text_image_pisa"] = Workload("text_image_pisa", 1, 24, 4352, 128, 128, "pisa",
                                     density=0.15, generator="block_centres",

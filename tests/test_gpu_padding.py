@@ -45,7 +45,7 @@ def _heads(x, heads):
 # d = 64 (mma.sync statistics kernel) and d = 128 (tcgen05 statistics kernel); the
 # second and the last case carry a one-token (timestep) block
 PRE_CASES = [
-    ("multimodal_dit", [0, 77, 127]),
+    ("multimodal_dit_padded", [0, 77, 127]),
     ("text_image_pisa", [0, 9, 23]),
     ("pad64_d128", [0, 1]),
 ]
@@ -164,7 +164,7 @@ def test_forward_masks_pad_keys(name, mode):
 def test_forward_pisa_over_the_padded_multimodal_mask_per_block_mode():
     """The fixed multimodal pattern (text blocks in every row, so the padded text block
     is exact everywhere) with the per-block first-order tail."""
-    w = synth.workloads()["multimodal_dit"]
+    w = synth.workloads()["multimodal_pisa_padded"]
     q, k, v = synth.make_qkv(w, seed=1)
     valid = w.valid_tokens()
     keep = orc.mask_dense(**w.mask)

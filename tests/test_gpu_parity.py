@@ -202,10 +202,12 @@ def test_forward_tiny_random_lists(mode):
     _forward_check(w, q, k, v, rp, ci, 1, mode, (kbar, vsum, Hbar))
 
 
-def test_forward_multimodal_fixed_mask_keep_or_drop():
-    """77 text tokens in two 64-blocks (13 real in the second): the 51 pad keys, filled
-    with large noise, must not reach any output row."""
-    w = synth.workloads()["multimodal_dit"]
+@pytest.mark.parametrize("name", ["multimodal_dit", "multimodal_dit_padded"])
+def test_forward_multimodal_fixed_mask_keep_or_drop(name):
+    """Without and with the token mask: in the padded workload the 77 text tokens fill
+    two 64-blocks (13 real in the second), and the 51 pad keys, filled with large noise,
+    must not reach any output row."""
+    w = synth.workloads()[name]
     q, k, v = synth.make_qkv(w)
     keep = orc.mask_dense(**w.mask)
     rp, ci = orc.dense_to_csr(keep)
@@ -213,11 +215,12 @@ def test_forward_multimodal_fixed_mask_keep_or_drop():
                    heads_idx=[0, 17, 63, 127], key_valid=w.valid_tokens())
 
 
-def test_forward_pisa_over_the_multimodal_fixed_mask():
+@pytest.mark.parametrize("name", ["multimodal_pisa", "multimodal_pisa_padded"])
+def test_forward_pisa_over_the_multimodal_fixed_mask(name):
     """PISA with S_i from the fixed multimodal pattern (one shared CSR list for every
     head) and U_i its complement: the blocks the mask drops enter through the Taylor tail
     instead of vanishing. The forward gets the oracle statistics, so the check isolates it."""
-    w = synth.workloads()["multimodal_dit"]
+    w = synth.workloads()[name]
     q, k, v = synth.make_qkv(w)
     keep = orc.mask_dense(**w.mask)
     rp, ci = orc.dense_to_csr(keep)
