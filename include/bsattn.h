@@ -40,7 +40,8 @@
  *     real-token count; a padded block is always computed exactly: bsa_route places it
  *     in every list, and bsa_forward in the PISA modes reports BSA_ERR_BAD_PADDING for a
  *     list that lacks one. Padded query rows are computed like any other row. Values
- *     outside 1..block report BSA_ERR_BAD_PADDING (and are clamped).
+ *     outside 1..block report BSA_ERR_BAD_PADDING (and are clamped). A key_valid
+ *     pointer that is not 4-byte aligned returns BSA_ERR_INVALID_ARG.
  */
 #ifndef BSATTN_H
 #define BSATTN_H
