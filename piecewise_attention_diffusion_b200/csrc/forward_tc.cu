@@ -259,7 +259,7 @@ struct Barriers {
   uint64_t kv_full[8], kv_empty[8];
   uint64_t q_full[kStreams];
   uint64_t s_full[kStreams], p_full[kStreams];
-  uint64_t o_final[kStreams], o_free[kStreams];
+  uint64_t o_final[kStreams], o_free[kStreams], o_staged[kStreams];
   uint64_t done;
 };
 
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
           const __grid_constant__ CUtensorMap tmVs, const __grid_constant__ CUtensorMap tmHb,
-          const Params p) {
+          const __grid_constant__ CUtensorMap tmO, const Params p) {
   using C = Cfg<D, BKV>;
   if (*p.flag) return;  // malformed lists: leave O untouched
 
@@ -289,6 +289,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       mbar_init(&bars.p_full[x], 128);
       mbar_init(&bars.o_final[x], 1);
       mbar_init(&bars.o_free[x], 128);
+      mbar_init(&bars.o_staged[x], 128);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(&bars.kv_full[i], 1);
@@ -457,13 +458,13 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         // PV(u) with P (bf16, TMEM) of tile u, then S(t): both operands' waits first, so
         // that the step's MMAs go out back to back
         const int u = s.t - 1;
-        if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag)) return false;
-        tc_fence_after();
         uint32_t v_addr, k_addr = 0;
         if (!wait_slot(v_addr)) return false;
         const uint32_t v_slot = last;
         const bool more = s.t < s.n;
         if (more && !wait_slot(k_addr)) return false;
+        if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag)) return false;
+        tc_fence_after();
         {
           const int kdim = u >= s.n_ex ? kChunk : BKV;
           const uint64_t b0 = smem_desc_sw128(v_addr, kdim * 128, 1024);
@@ -719,8 +720,12 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      // every MMA of this item has completed: Q's buffer is free for the next item
-      if (q_loader && stream_item(k + 1, x) < p.n_items) {
+      // every MMA of this item has completed: Q's buffer is free. With full 128-row tiles
+      // it first stages this tile's output for one TMA store (coalesced, asynchronous) and
+      // takes the next Q after the store has read it; otherwise the next Q is loaded now
+      // and every row is stored directly.
+      const bool tma_out = p.qbox == kBQ;
+      if (!tma_out && q_loader && stream_item(k + 1, x) < p.n_items) {
         load_q(stream_item(k + 1, x));
         ++q_issued;
       }
@@ -750,11 +755,38 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           }
           packed[e / 2] = pack_bf16x2(a0 * inv_l, a1 * inv_l);
         }
-        if (write) {
+        if (tma_out) {
+          // 128-byte swizzle of the Q layout: 16-byte chunk j of row r sits at j ^ (r % 8)
+          const int j = (c % 64) / 8;
+          unsigned char* rp_s = sq + (c / 64) * (kBQ * 128) + row * 128;
+          *reinterpret_cast<uint4*>(rp_s + ((j ^ (row & 7)) * 16)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          *reinterpret_cast<uint4*>(rp_s + (((j + 1) ^ (row & 7)) * 16)) =
+              make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        } else if (write) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
+      }
+      if (tma_out) {
+        fence_proxy_async_smem();
+        mbar_arrive(&bars.o_staged[x]);  // this row is staged
+        bool staged = true;
+        if (q_loader) {
+          staged = mbar_wait(&bars.o_staged[x], k & 1, abort_flag);
+          if (staged) {
+            tma_store_4d(&tmO, sq, 0, qt * kBQ, 0, bh);  // rows past L are not written
+            bulk_commit_group();
+            bulk_wait_read_all();
+            if (stream_item(k + 1, x) < p.n_items) {
+              load_q(stream_item(k + 1, x));
+              ++q_issued;
+            }
+          }
+        }
+        ok = __all_sync(0xffffffffu, staged);
+        if (!ok) break;
       }
       if (write && p.lse)
         p.lse[(size_t)bh * p.L + row_g] =
@@ -763,6 +795,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       mbar_arrive(&bars.o_free[x]);
       tiles += n;
     }
+    if (q_loader) bulk_wait_all();  // this stream's output stores have completed
     if (!ok && q_loader && q_issued > 0) {
       // drain this stream's last Q copy (bounded) before the CTA exits
       const uint64_t t0 = globaltimer_ns();
@@ -861,12 +894,15 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   using C = Cfg<D, BKV>;
   const Shape& s = a.s;
   const int BH = s.BH(), M = s.M();
-  CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmHb;
+  CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmHb, tmO;
   const int qbox = s.L < kBQ ? s.L : kBQ;
   const int Mp = ceil_div(M, kChunk) * kChunk;
   bool ok = make_map(&tmQ, a.Q, D, s.L, BH, qbox, qbox == kBQ) &&
             make_map(&tmK, a.K, D, s.L, BH, BKV) &&
             make_map(&tmV, a.V, D, s.L, BH, BKV);
+  // the output map (128-row boxes) is used only when every query tile is 128 rows
+  if (qbox == kBQ) ok = ok && make_map(&tmO, a.O, D, s.L, BH, kBQ);
+  else tmO = tmQ;
   if (a.mode == BSA_MODE_PISA) {
     ok = ok && make_map(&tmKb, kb16, D, Mp, BH, kChunk) && make_map(&tmVs, vs16, D, Mp, BH, kChunk) &&
          make_map(&tmHb, hb16, D, D, BH, D);
@@ -904,7 +940,8 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   if (fa.numRegs * kThreads < 128 * kRegsControl + 128 * kStreams * kRegsSoftmax)
     return cudaErrorInvalidConfiguration;
   const int grid = min(p.n_items, sm_count());
-  k_forward<D, BKV, kLinear><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, p);
+  k_forward<D, BKV, kLinear><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, tmO,
+                                                                p);
   return cudaGetLastError();
 }
 
