@@ -11,9 +11,10 @@
 // One CTA per (head, 8 query blocks), one warp per query block:
 //   1. pooled query: the warp streams its block of Q with 16-byte loads (the only HBM
 //      stream of the call) and reduces the columns;
-//   2. scores: thread t takes centroid j = t (looping when M > 256), reads its row once
-//      per CTA (16-byte loads from L2) and dots it with the CTA's 8 pooled queries, which
-//      every thread reads from the same shared-memory words (broadcast);
+//   2. scores: thread t takes centroid j = t (looping when M > 256; with M <= 128 two
+//      threads share a centroid, half of d each, and add across the pair), reads its row
+//      once per CTA (16-byte loads from L2) and dots it with the CTA's 8 pooled queries,
+//      which every thread reads from the same shared-memory words (broadcast);
 //   3. softmax over the M blocks plus the normalised covariance term;
 //   4. exact top-k: the k-th largest score is found by a radix select on the float bit
 //      patterns (scores are >= 0, so the bit patterns order like the values), ties at
@@ -112,13 +113,20 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   // 16-byte loads when the caller's kbar allows them (each head's slice then does too,
   // since M * D * 4 is a multiple of 16)
   const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
-  for (int j = threadIdx.x; j < M; j += kThreads) {
+  // with at most kThreads / 2 centroids two threads share one (half of d each)
+  const int split = 2 * M <= kThreads ? 2 : 1;
+  const int total = M * split;
+  for (int base = warp * 32; base < total; base += kThreads) {
+    const int jj = base + lane;
+    const bool valid = jj < total;
+    const int j = valid ? jj / split : 0, part = jj % split;
     float acc[kWarps];
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) acc[w] = 0.f;
     const float* kr = kb + (size_t)j * D;
+    const int cb = part * (D / split), ce = cb + D / split;
 #pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
+    for (int c = cb; c < ce; c += 4) {
       float4 kv;
       if (vec) {
         kv = __ldg(reinterpret_cast<const float4*>(kr + c));
@@ -131,8 +139,14 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
         acc[w] = fmaf(qv.w, kv.w, fmaf(qv.z, kv.z, fmaf(qv.y, kv.y, fmaf(qv.x, kv.x, acc[w]))));
       }
     }
+    if (split == 2) {
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) s_sc[w * M + j] = scale * acc[w];
+      for (int w = 0; w < kWarps; ++w) acc[w] += __shfl_xor_sync(0xffffffffu, acc[w], 1);
+    }
+    if (valid && part == 0) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) s_sc[w * M + j] = scale * acc[w];
+    }
   }
   __syncthreads();
   __syncwarp();
