@@ -61,20 +61,35 @@ struct Params {
   int32_t* status;
 };
 
-// The blocks this CTA processes, in order: the contiguous range [u0, u1) of the pass.
+// The blocks this CTA processes, in order: the contiguous range [u0, u1) of the pass,
+// ascending in the statistics pass and descending in the norm pass, so that the norm pass
+// starts on the blocks the statistics pass read last (still in L2).
 // A head segment is the run of the range's blocks that belong to one head.
 struct BlockIter {
-  int u, u1, j, bh, M;
+  int u, u0, u1, j, bh, M;
+  bool down;
   __device__ __forceinline__ void init(const Params& p) {
     M = p.M;
-    u = blockIdx.x * p.per_cta;
-    u1 = min(p.n_units, u + p.per_cta);
+    u0 = blockIdx.x * p.per_cta;
+    u1 = min(p.n_units, u0 + p.per_cta);
+    down = !p.stats;
+    u = down ? u1 - 1 : u0;
     bh = u / M;
     j = u % M;
   }
-  __device__ __forceinline__ bool valid() const { return u < u1; }
-  // advance to the next block; returns true when a head segment just ended
+  __device__ __forceinline__ bool valid() const { return down ? u >= u0 : u < u1; }
+  // advance to the next block; returns true when a head segment just ended (used by
+  // the ascending statistics pass)
   __device__ __forceinline__ bool next() {
+    if (down) {
+      --u;
+      if (--j < 0) {
+        j = M - 1;
+        --bh;
+        return true;
+      }
+      return u < u0;
+    }
     ++u;
     ++j;
     if (j == M) {
