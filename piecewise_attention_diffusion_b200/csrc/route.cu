@@ -180,12 +180,31 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
 
   // 4. k-th largest key (bit pattern of a non-negative float) by radix select
   uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    int cnt = 0;
-    for (int j = lane; j < M; j += 32) cnt += __float_as_uint(sc[j]) >= cand ? 1 : 0;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= k_top) T = cand;
+  if (M <= 128) {
+    // up to 4 keys per lane, held in registers for the 32 passes (absent keys 0: never
+    // counted, every candidate has a bit set)
+    uint32_t key[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = lane + 32 * q;
+      key[q] = j < M ? __float_as_uint(sc[j]) : 0u;
+    }
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) cnt += key[q] >= cand ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= k_top) T = cand;
+    }
+  } else {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+      for (int j = lane; j < M; j += 32) cnt += __float_as_uint(sc[j]) >= cand ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= k_top) T = cand;
+    }
   }
   int greater = 0;
   for (int j = lane; j < M; j += 32) greater += __float_as_uint(sc[j]) > T ? 1 : 0;
