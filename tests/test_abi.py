@@ -27,6 +27,23 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(so, name), name
 
 
+def test_header_status_and_mode_values_match_binding():
+    with open(os.path.join(ROOT, "include", "bsattn.h")) as f:
+        src = f.read()
+    codes = dict((n, int(v)) for n, v in re.findall(r"\b(BSA_(?:OK|ERR_\w+))\s*=\s*(\d+)", src))
+    assert codes == {"BSA_OK": b.OK, "BSA_ERR_INVALID_ARG": b.ERR_INVALID_ARG,
+                     "BSA_ERR_UNSUPPORTED": b.ERR_UNSUPPORTED, "BSA_ERR_CUDA": b.ERR_CUDA,
+                     "BSA_ERR_BAD_CSR": b.ERR_BAD_CSR, "BSA_ERR_TIMEOUT": b.ERR_TIMEOUT,
+                     "BSA_ERR_WORKSPACE": b.ERR_WORKSPACE, "BSA_ERR_CAPACITY": b.ERR_CAPACITY,
+                     "BSA_ERR_SCRATCH_LIMIT": b.ERR_SCRATCH_LIMIT,
+                     "BSA_ERR_BAD_PADDING": b.ERR_BAD_PADDING}
+    modes = dict((n, int(v)) for n, v in re.findall(r"\b(BSA_MODE_\w+)\s*=\s*(\d+)", src))
+    assert modes == {"BSA_MODE_KEEP_OR_DROP": b.MODE_KEEP_OR_DROP, "BSA_MODE_PISA": b.MODE_PISA,
+                     "BSA_MODE_PISA_BLOCK": b.MODE_PISA_BLOCK}
+    for code in codes.values():
+        assert b.status_string(code) != "BSA_UNKNOWN_STATUS"
+
+
 def test_status_strings_and_version():
     assert b.bsa_version() >= 100
     assert b.status_string(b.OK) == "BSA_OK"
@@ -118,6 +135,14 @@ def test_route_and_precompute_reject_bad_arguments():
         b.ERR_INVALID_ARG
     assert pc(p, p, 1, 2, 512, 64, 64, odd, p, p, p, p, None, p, 1 << 30, None, None) == \
         b.ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_misaligned_key_valid():
+    p = _fake()
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    rc = b.lib().bsa_forward_noalloc(p, p, p, 1, 2, 512, 64, 64, odd, p, p, 16, 0, 0, None, None,
+                                     None, 0.0, p, None, None, None)
+    assert rc == b.ERR_INVALID_ARG
 
 
 def test_build_mask_rejects_bad_arguments():
