@@ -153,3 +153,20 @@ def test_build_mask_rejects_bad_arguments():
     bad = b.MaskDesc(2, 4, 0, 1, 16, 0)
     assert b.lib().bsa_build_mask(ctypes.byref(bad), p, p, 324, None, None) == \
         b.ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    """There is no CPU path: every wrapper refuses tensors that are not on a CUDA device
+    before anything is launched."""
+    import torch
+    q = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    f32 = dict(dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.forward(q, q, q, 64, torch.zeros(5, dtype=torch.int32),
+                  torch.zeros(8, dtype=torch.int32), 0, b.MODE_KEEP_OR_DROP, ws=q)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.bsa_route(q, torch.zeros(2, 4, 64, **f32), torch.zeros(2, 4, **f32), 64, 2, 1.0, 0.0,
+                    torch.zeros(10, dtype=torch.int32), torch.zeros(16, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        b.bsa_precompute(q, q, 64, torch.zeros(2, 4, 64, **f32), torch.zeros(2, 4, 64, **f32),
+                         torch.zeros(2, 64, 64, **f32), torch.zeros(2, 4, **f32))
