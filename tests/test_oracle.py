@@ -477,3 +477,35 @@ def test_routing_places_every_padded_block_in_every_list():
             assert 0 in row and 3 in row and row == sorted(row) and len(row) == kk
     with pytest.raises(ValueError):
         orc.route_head(q, kbar, Mn, block, 1, 1.0, s, key_valid=valid)
+
+
+def test_pisa_padded_block_in_the_tail_weighs_its_real_tokens():
+    """A padded block left in U_i (the oracle accepts such lists; the GPU refuses them).
+    When every block's real keys are one vector c_j, the zeroth-order term of block j
+    is exact: sum over its real keys of e^{s q.c_j} v_n = alpha_tj vsum_j and the
+    denominator gains (real tokens) x alpha_tj, while H_j = 0 and Hbar = 0. PISA then
+    equals softmax attention over the real keys only, whatever the lists; a tail
+    weight of B instead of the real-token count, or pad rows in the value sum, breaks
+    the equality."""
+    q, k, v, valid, block = _padded_case(30)
+    M = q.shape[0] // block
+    s = 1 / math.sqrt(q.shape[1])
+    centres = _rng(31).standard_normal((M, k.shape[1]))
+    k = np.array(k, copy=True)
+    for j in range(M):
+        k[j * block:j * block + valid[j]] = centres[j]
+    k, v = (_garbage(x, valid, block, 32 + n) for n, x in enumerate((k, v)))
+    kbar, vsum, H, Hbar, Mn = orc.precompute_head(k, v, block, key_valid=valid)
+    assert np.abs(Hbar).max() < 1e-12
+    # lists that leave both padded blocks (0 and 3) out of some rows
+    keep = np.zeros((M, M), dtype=bool)
+    keep[:, 1] = True
+    keep[0, 0] = keep[2, 3] = keep[4, 5] = True
+    rp, ci = orc.dense_to_csr(keep)
+    assert any(0 not in ci[rp[i]:rp[i + 1]] for i in range(M))
+    assert any(3 not in ci[rp[i]:rp[i + 1]] for i in range(M))
+    out, lse = orc.pisa_head(q, k, v, rp, ci, block, s, kbar, vsum, Hbar, key_valid=valid)
+    allowed = np.zeros((q.shape[0], q.shape[0]), dtype=bool)
+    for j in range(M):
+        allowed[:, j * block:j * block + valid[j]] = True
+    np.testing.assert_allclose(out, _masked_sdpa(q, k, v, s, allowed), rtol=1e-10, atol=1e-12)
