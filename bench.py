@@ -279,91 +279,178 @@ def oracle_sample(w, k_top, heads_sample: int, seed: int = 0) -> dict:
 
 
 # --------------------------------------------------------------------- our arm
-def run_ours(args, w, world, rank, local):
-    from piecewise_attention_diffusion_b200 import bsattn as b
+L2_BYTES = 126 * 2 ** 20
+# the forward of these workloads is reported beside the headline: the long-sequence
+# sweep's 4K, 16K and 32K points at 12.5% density in both modes, and the other configs
+SWEEP_WORKLOADS = ("sweep_L4096_d125_pisa", "sweep_L4096_d125_keep_or_drop",
+                   "sweep_L16384_d125_pisa", "sweep_L16384_d125_keep_or_drop",
+                   "sweep_L32768_d125_pisa", "sweep_L32768_d125_keep_or_drop",
+                   "tiny_pisa", "multimodal_dit", "image_pisa")
 
+
+def input_bytes(w) -> int:
+    """Bytes of Q, K and V (bf16) of a workload."""
+    return 3 * w.batch * w.heads * w.seq_len * w.head_dim * 2
+
+
+def needs_flush(w) -> bool:
+    """Inputs that fit twice in L2 are timed with an L2 flush before every step."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
+def config_of(w, world: int) -> dict:
+    """The workload as both arms name it (identical keys and values)."""
+    k_top = 0 if w.mask else w.top_k()
+    l2 = (f"inputs larger than L2 (Q+K+V = {input_bytes(w) / 1e6:.0f} MB)" if not needs_flush(w)
+          else f"L2 flushed before every step (Q+K+V = {input_bytes(w) / 1e6:.0f} MB)")
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq_len,
+            "head_dim": w.head_dim, "block": w.block, "mode": w.mode, "density": w.density,
+            "k_top": None if w.mask else k_top, "lambda": LAMBDA,
+            "lists": "fixed multimodal mask (shared)" if w.mask else "bsa_route top-k",
+            "real_tokens_per_block": w.valid_tokens() if w.key_valid else None,
+            "parallelism": f"replicas x{world}", "l2": l2}
+
+
+class Path:
+    """Device buffers and the launch sequence of one step of a workload:
+    bsa_precompute -> bsa_route -> bsa_forward (the statistics and routing are skipped
+    where the workload does not need them)."""
+
+    def __init__(self, w, q, k, v, dev):
+        from piecewise_attention_diffusion_b200 import bsattn as b
+        self.b, self.w, self.dev = b, w, dev
+        self.k_top = 0 if w.mask else w.top_k()  # a fixed mask has no top-k
+        BH, M, L, d = w.batch * w.heads, w.n_blocks, w.seq_len, w.head_dim
+        self.qd, self.kd, self.vd = q.to(dev), k.to(dev), v.to(dev)
+        self.st = torch.zeros(1, dtype=torch.int32, device=dev)
+        # real tokens per block (token padding), a constant of the workload like its mask
+        self.kv = None if not w.key_valid else torch.tensor(w.valid_tokens(), dtype=torch.int32,
+                                                            device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.stats = dict(kbar=torch.empty(BH, M, d, **f32), vsum=torch.empty(BH, M, d, **f32),
+                          Hbar=torch.empty(BH, d, d, **f32), Mnorm=torch.empty(BH, M, **f32))
+        if w.mask:
+            # fixed multimodal pattern: one shared list for every head, built once
+            self.rp, self.ci = b.build_mask(b.MaskDesc(**w.mask), device=dev, status=self.st)
+            torch.cuda.synchronize()
+            self.row_lens = np.diff(self.rp.cpu().numpy()).tolist()
+            self.per_head = 0
+        else:
+            self.rp = torch.empty(BH * (M + 1), dtype=torch.int32, device=dev)
+            self.ci = torch.empty(BH * M * self.k_top, dtype=torch.int32, device=dev)
+            self.row_lens = None
+            self.per_head = 1
+        self.O = torch.empty_like(self.qd)
+        self.ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
+        self.ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
+        self.mode = {"pisa": b.MODE_PISA, "pisa_block": b.MODE_PISA_BLOCK}.get(
+            w.mode, b.MODE_KEEP_OR_DROP)
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, qx=None, kx=None, vx=None, ev=None, out=None):
+        b, w, st, s = self.b, self.w, self.st, self.stats
+        qx = self.qd if qx is None else qx
+        kx = self.kd if kx is None else kx
+        vx = self.vd if vx is None else vx
+        if ev:
+            ev[0].record(self.stream)
+        if needs_precompute(w):
+            b.bsa_precompute(kx, vx, w.block, s["kbar"], s["vsum"], s["Hbar"], s["Mnorm"], None,
+                             self.ws_p, st, key_valid=self.kv)
+        if ev:
+            ev[1].record(self.stream)
+        if not w.mask:
+            b.bsa_route(qx, s["kbar"], s["Mnorm"], w.block, self.k_top, LAMBDA, 0.0, self.rp,
+                        self.ci, None, st, key_valid=self.kv)
+        if ev:
+            ev[2].record(self.stream)
+        b.bsa_forward(qx, kx, vx, w.block, self.rp, self.ci, self.per_head, self.mode,
+                      s["kbar"], s["vsum"], s["Hbar"], 0.0, self.O if out is None else out,
+                      None, self.ws_f, st, key_valid=self.kv)
+        if ev:
+            ev[3].record(self.stream)
+
+    def check_status(self):
+        if self.st.item() != 0:
+            raise RuntimeError(f"device status {self.b.status_string(self.st.item())}")
+
+    def measure(self, steps: int, warmup: int, world: int = 1) -> dict:
+        """Time `steps` steps after `warmup` untimed ones, CUDA events on the launching
+        stream around every phase of every step, max over ranks. Workloads whose inputs
+        fit in L2 get an L2 flush (a 256 MB write) before every step, outside the
+        events; the step time is then the sum of the per-step event spans."""
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=self.dev) \
+            if needs_flush(self.w) else None
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        self.check_status()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = time.time()
+        t_start.record(self.stream)
+        for n in range(steps):
+            if flush is not None:
+                flush.zero_()
+            self.step(ev=evs[n])
+        t_end.record(self.stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        barrier(world)
+        self.check_status()
+        span = lambda a, z: sum(e[a].elapsed_time(e[z]) for e in evs) / steps
+        ms_step = t_start.elapsed_time(t_end) / steps if flush is None else span(0, 3)
+        F_fwd = forward_flops(self.w, self.k_top, self.w.mode, self.row_lens)
+        F_step = F_fwd + (precompute_flops(self.w) if needs_precompute(self.w) else 0.0) \
+            + (0.0 if self.w.mask else route_flops(self.w))
+        return {"ms_step": max_over_ranks(ms_step, world),
+                "fwd_ms": max_over_ranks(span(2, 3), world),
+                "pre_ms": span(0, 1), "route_ms": span(1, 2), "F_fwd": F_fwd, "F_step": F_step,
+                "t0": t0, "t1": t1, "flushed": flush is not None}
+
+
+def run_sweep(args, world, rank, local) -> dict:
+    """Forward (and step) numbers of the other workloads, measured in the same run: per
+    workload its own inputs, 3 warm-up steps and `--sweep-steps` timed steps."""
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    out, cache = {}, {}
+    for name in SWEEP_WORKLOADS:
+        w = synth.workloads()[name]
+        key = (w.seq_len, w.heads, w.batch, w.head_dim, w.block, w.generator, w.grid,
+               w.key_valid)
+        if key not in cache:
+            cache.clear()
+            cache[key] = synth.make_qkv(w, seed=args.seed + rank)
+        path = Path(w, *cache[key], dev)
+        m = path.measure(args.sweep_steps, 3, world)
+        tf = m["F_fwd"] / (m["fwd_ms"] * 1e-3) / 1e12
+        out[name] = {"seq_len": w.seq_len, "heads": w.heads, "mode": w.mode,
+                     "density": w.density, "k_top": None if w.mask else path.k_top,
+                     "forward_ms": round(m["fwd_ms"], 4), "forward_tflops": round(tf, 2),
+                     "frac": round(tf / pk["bf16_tflops"], 4),
+                     "precompute_ms": round(m["pre_ms"], 4), "route_ms": round(m["route_ms"], 4),
+                     "step_ms": round(m["ms_step"], 4), "forward_gflop": round(m["F_fwd"] / 1e9, 3),
+                     "l2": "flushed before every step" if m["flushed"] else "inputs larger than L2"}
+        del path
+    return {"steps": args.sweep_steps, "warmup": 3, "peak_tflops": pk["bf16_tflops"],
+            "peak_source": f"{pk['source']} bf16_tflops (burst)", "points": out}
+
+
+def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    k_top = 0 if w.mask else w.top_k()  # a fixed mask has no top-k
-    BH, M, L, d = w.batch * w.heads, w.n_blocks, w.seq_len, w.head_dim
     q, k, v = synth.make_qkv(w, seed=args.seed + rank)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    st = torch.zeros(1, dtype=torch.int32, device=dev)
-    # real tokens per block (token padding), a constant of the workload like its mask
-    kv = None if not w.key_valid else torch.tensor(w.valid_tokens(), dtype=torch.int32,
-                                                   device=dev)
-    f32 = dict(dtype=torch.float32, device=dev)
-    stats = dict(kbar=torch.empty(BH, M, d, **f32), vsum=torch.empty(BH, M, d, **f32),
-                 Hbar=torch.empty(BH, d, d, **f32), Mnorm=torch.empty(BH, M, **f32))
-    if w.mask:
-        # fixed multimodal pattern: one shared list for every head, built once
-        desc = b.MaskDesc(**w.mask)
-        rp, ci = b.build_mask(desc, device=dev, status=st)
-        torch.cuda.synchronize()
-        row_lens = np.diff(rp.cpu().numpy()).tolist()
-        per_head = 0
-    else:
-        rp = torch.empty(BH * (M + 1), dtype=torch.int32, device=dev)
-        ci = torch.empty(BH * M * k_top, dtype=torch.int32, device=dev)
-        row_lens = None
-        per_head = 1
-    O = torch.empty_like(qd)
-    ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
-    ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
-    mode = {"pisa": b.MODE_PISA, "pisa_block": b.MODE_PISA_BLOCK}.get(w.mode, b.MODE_KEEP_OR_DROP)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(qx, kx, vx, ev=None, out=None):
-        if ev:
-            ev[0].record(stream)
-        if needs_precompute(w):
-            b.bsa_precompute(kx, vx, w.block, stats["kbar"], stats["vsum"], stats["Hbar"],
-                             stats["Mnorm"], None, ws_p, st, key_valid=kv)
-        if ev:
-            ev[1].record(stream)
-        if not w.mask:
-            b.bsa_route(qx, stats["kbar"], stats["Mnorm"], w.block, k_top, LAMBDA, 0.0, rp, ci,
-                        None, st, key_valid=kv)
-        if ev:
-            ev[2].record(stream)
-        b.bsa_forward(qx, kx, vx, w.block, rp, ci, per_head, mode, stats["kbar"],
-                      stats["vsum"], stats["Hbar"], 0.0, O if out is None else out, None, ws_f, st,
-                      key_valid=kv)
-        if ev:
-            ev[3].record(stream)
+    path = Path(w, q, k, v, dev)
+    BH, L, d = w.batch * w.heads, w.seq_len, w.head_dim
 
     clk = ClockSampler(local).start()
     time.sleep(0.5)  # let nvidia-smi start sampling before the GPU work begins
-    for _ in range(args.warmup):
-        step(qd, kd, vd)
-    torch.cuda.synchronize()
-    if st.item() != 0:
-        raise RuntimeError(f"device status {b.status_string(st.item())}")
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    clk.t0 = time.time()
-    t_start.record(stream)
-    for s in range(args.steps):
-        step(qd, kd, vd, evs[s])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    clk.t1 = time.time()
-    barrier(world)
-    ms_total = t_start.elapsed_time(t_end)
-    pre_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    route_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    fwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    ms_step = max_over_ranks(ms_total / args.steps, world)
-    fwd_ms = max_over_ranks(fwd_ms, world)
-    if st.item() != 0:
-        raise RuntimeError(f"device status {b.status_string(st.item())}")
-
-    F_fwd = forward_flops(w, k_top, w.mode, row_lens)
-    F_step = F_fwd + (precompute_flops(w) if needs_precompute(w) else 0.0) \
-        + (0.0 if w.mask else route_flops(w))
+    m = path.measure(args.steps, args.warmup, world)
+    clk.t0, clk.t1 = m["t0"], m["t1"]
+    ms_step, fwd_ms, F_fwd, F_step = m["ms_step"], m["fwd_ms"], m["F_fwd"], m["F_step"]
     value = replica_value(F_step, ms_step, world)
     pk = peaks()
     achieved = F_fwd / (fwd_ms * 1e-3) / 1e12
@@ -372,9 +459,12 @@ def run_ours(args, w, world, rank, local):
     # copies its Q, K, V in and its O out; the steps are pipelined as a serving loop would
     # run them: two device buffer sets, the copies in on one stream and out on another,
     # so that step i's copies overlap step i-1's compute and each other (PCIe is full
-    # duplex). Events order each buffer's reuse.
+    # duplex). Events order each buffer's reuse. The latency of one step run alone (its
+    # copies and compute in sequence on one stream) is reported beside it.
     e2e = None
     if not args.no_e2e:
+        stream = path.stream
+        qd, kd, vd, O = path.qd, path.kd, path.vd, path.O
         qh, kh, vh = (x.pin_memory() for x in (q, k, v))
         Oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
         sets = [(qd, kd, vd, O),
@@ -400,7 +490,7 @@ def run_ours(args, w, world, rank, local):
                 stream.wait_event(in_done[x])
                 if i >= 2:
                     stream.wait_event(out_done[x])     # step i-2's output has been read
-                step(qx, kx, vx, out=ox)
+                path.step(qx, kx, vx, out=ox)
                 comp_done[x].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(comp_done[x])
@@ -419,8 +509,26 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / args.steps, world)
+        # one step at a time: copies in, the path, copy out, all on the launching stream
+        n_serial = min(args.steps, 10)
+        s_s, s_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        s_s.record(stream)
+        for _ in range(n_serial):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            path.step()
+            Oh.copy_(O, non_blocking=True)
+        s_e.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        serial_ms = max_over_ranks(s_s.elapsed_time(s_e) / n_serial, world)
         e2e = {"value": round(replica_value(F_step, e2e_ms, world), 3), "unit": "TFLOP/s",
-               "ms_per_step": round(e2e_ms, 4),
+               "ms_per_step": round(e2e_ms, 4), "pipelined": True, "depth": 2,
+               "serial_ms_per_step": round(serial_ms, 4),
+               "serial_value": round(replica_value(F_step, serial_ms, world), 3),
                "h2d_bytes_per_step": int(3 * q.numel() * 2),
                "d2h_bytes_per_step": int(O.numel() * 2)}
 
@@ -431,15 +539,9 @@ def run_ours(args, w, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: Q ~ N(0,1); K, V: " + GENERATOR_TEXT[w.generator] + ")",
-        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": L,
-                   "head_dim": d, "block": w.block, "mode": w.mode, "density": w.density,
-                   "k_top": None if w.mask else k_top, "lambda": LAMBDA,
-                   "lists": "fixed multimodal mask (shared)" if w.mask else "bsa_route top-k",
-                   "real_tokens_per_block": w.valid_tokens() if w.key_valid else None,
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2 (Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB)"},
+        "config": config_of(w, world),
         "forward_ms": round(fwd_ms, 4), "forward_tflops": round(achieved, 3),
-        "precompute_ms": round(pre_ms, 4), "route_ms": round(route_ms, 4),
+        "precompute_ms": round(m["pre_ms"], 4), "route_ms": round(m["route_ms"], 4),
         "forward_gflop": round(F_fwd / 1e9, 3),
         "dense_equiv_tflops": round(4.0 * BH * L * L * d / (fwd_ms * 1e-3) / 1e12, 3),
         "roofline": {"kernel": "bsa_forward", "bound": "tensor", "achieved": round(achieved, 3),
@@ -453,7 +555,11 @@ def run_ours(args, w, world, rank, local):
     }
     if e2e:
         line["e2e"] = e2e
+    del path
+    if not args.no_sweep:
+        line["sweep"] = run_sweep(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu:
+        k_top = 0 if w.mask else w.top_k()
         cs = oracle_sample(w, k_top, args.cpu_heads, args.seed)
         line["cpu_baseline"] = {"value": round(F_step / cs["seconds_full_est"] / 1e12, 6),
                                 "unit": "TFLOP/s", "cores": cs["cores"], "kind": "oracle",
@@ -488,10 +594,7 @@ def run_reference(args, w, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (same generator and seed)",
-            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads,
-                       "seq_len": w.seq_len, "head_dim": w.head_dim, "block": w.block,
-                       "mode": w.mode, "density": w.density, "k_top": k_top,
-                       "lambda": LAMBDA, "parallelism": "host cores"},
+            "config": config_of(w, world),
             "cpu_baseline": cpu,
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -511,6 +614,9 @@ def main():
     ap.add_argument("--ref-heads", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-workload forward numbers reported beside the headline")
+    ap.add_argument("--sweep-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

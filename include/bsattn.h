@@ -225,9 +225,9 @@ BSA_API bsa_status bsa_forward(const void* Q, const void* K, const void* V, int3
  * the same result; its scratch is one __device__ array of BSA_NOALLOC_SCRATCH_BYTES
  * inside the library, which every GPU that loads the library keeps until the process
  * exits. It calls no allocating routine.
- *   - The scratch address is looked up on the first call made on each device (with that
- *     device current, and the stream on that device); make that first call before any
- *     stream capture.
+ *   - The scratch address is looked up on the current device at every call (the device
+ *     of the stream); the first call on a device may load the library's device code, so
+ *     make it before any stream capture.
  *   - Every call shares the one array (per device) and leaves its contents behind; calls
  *     whose kernels overlap on the GPU (different streams or host threads) race on it,
  *     so serialise them.
@@ -252,6 +252,26 @@ BSA_API bsa_status bsa_forward_noalloc(const void* Q, const void* K, const void*
  *   timeout_ns  1 .. 10^10 (10 s); status: device int32, written with BSA_ERR_TIMEOUT.
  * Returns BSA_ERR_INVALID_ARG for a null status or a limit out of range. */
 BSA_API bsa_status bsa_selftest_wait_timeout(int64_t timeout_ns, int32_t* status, void* stream);
+
+/* bsa_selftest_forward_timeout — the attention kernel's own abort path, run without a fault.
+ * (No counterpart in the pages.) The same launch sequence as bsa_forward (per-head lists,
+ * no token padding, default scale, no lse), with every bounded wait of the attention
+ * kernel limited to wait_ns instead of its 2 s default. With a limit far below the time
+ * the kernel's copies and MMAs take, a wait runs out while TMA copies and tensor-core work
+ * are in flight: the CTA raises its abort flag, every role leaves its loop, the producer
+ * drains its copies, the MMA thread waits for its issued MMAs, TMEM is freed and
+ * BSA_ERR_TIMEOUT is written to *status. O is then partly written (unspecified); the
+ * context stays usable.
+ *   wait_ns  1 .. 10^10; status: device int32 the caller zeroes (required); other
+ *            arguments as bsa_forward. */
+BSA_API bsa_status bsa_selftest_forward_timeout(const void* Q, const void* K, const void* V,
+                                                int32_t Bt, int32_t H, int32_t L, int32_t d,
+                                                int32_t block, const int32_t* row_ptr,
+                                                const int32_t* col_idx, int64_t nnz_total,
+                                                int32_t mode, const float* kbar,
+                                                const float* vsum, const float* Hbar, void* O,
+                                                void* workspace, size_t ws_bytes,
+                                                int64_t wait_ns, int32_t* status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -29,7 +29,7 @@ CALL_BUILD_MASK, CALL_PRECOMPUTE, CALL_ROUTE, CALL_FORWARD = 0, 1, 2, 3
 # Every symbol include/bsattn.h declares, in header order.
 EXPORTS = ("bsa_version", "bsa_status_string", "bsa_mask_blocks", "bsa_workspace_bytes",
            "bsa_build_mask", "bsa_precompute", "bsa_route", "bsa_forward",
-           "bsa_forward_noalloc", "bsa_selftest_wait_timeout")
+           "bsa_forward_noalloc", "bsa_selftest_wait_timeout", "bsa_selftest_forward_timeout")
 
 
 class BsaError(RuntimeError):
@@ -62,6 +62,9 @@ _SIGS = {
     "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                    _i64, _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp]),
     "bsa_selftest_wait_timeout": (_i32, [_i64, _vp, _vp]),
+    "bsa_selftest_forward_timeout": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                                            _vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _sz,
+                                            _i64, _vp, _vp]),
 }
 
 
@@ -210,7 +213,8 @@ def bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum
         _need(lse, torch.float32, "lse", (Bt * H, L))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().bsa_forward(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block,
-                             _key_valid(key_valid, L, block), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), int(csr_per_head), int(mode),
+                             _key_valid(key_valid, L, block), _ptr(row_ptr), _ptr(col_idx),
+                             col_idx.numel(), int(csr_per_head), int(mode),
                              _ptr(kbar), _ptr(vsum), _ptr(Hbar), float(scale), _ptr(O),
                              _ptr(lse), _ptr(workspace), ws_bytes, _ptr(status),
                              _stream(stream)), "bsa_forward")
@@ -234,7 +238,8 @@ def bsa_forward_noalloc(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kb
     if lse is not None:
         _need(lse, torch.float32, "lse", (Bt * H, L))
     _check(lib().bsa_forward_noalloc(_ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block,
-                                     _key_valid(key_valid, L, block), _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                     _key_valid(key_valid, L, block), _ptr(row_ptr),
+                                     _ptr(col_idx), col_idx.numel(),
                                      int(csr_per_head), int(mode), _ptr(kbar), _ptr(vsum),
                                      _ptr(Hbar), float(scale), _ptr(O), _ptr(lse),
                                      _ptr(status), _stream(stream)), "bsa_forward_noalloc")
@@ -246,6 +251,25 @@ def bsa_selftest_wait_timeout(timeout_ns, status, stream=None):
     _need(status, torch.int32, "status")
     _check(lib().bsa_selftest_wait_timeout(int(timeout_ns), _ptr(status), _stream(stream)),
            "bsa_selftest_wait_timeout")
+
+
+def bsa_selftest_forward_timeout(Q, K, V, block, row_ptr, col_idx, mode, kbar, vsum, Hbar, O,
+                                 workspace, wait_ns, status, stream=None):
+    """bsa_forward (per-head lists) with every bounded wait of the attention kernel limited
+    to wait_ns: the kernel's abort and drain path, reported as BSA_ERR_TIMEOUT in `status`."""
+    Bt, H, L, d = _bhld(Q, "Q")
+    _need(K, torch.bfloat16, "K", Q.shape)
+    _need(V, torch.bfloat16, "V", Q.shape)
+    _need(O, torch.bfloat16, "O", Q.shape)
+    _need(row_ptr, torch.int32, "row_ptr")
+    _need(col_idx, torch.int32, "col_idx")
+    _need(status, torch.int32, "status")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().bsa_selftest_forward_timeout(
+        _ptr(Q), _ptr(K), _ptr(V), Bt, H, L, d, block, _ptr(row_ptr), _ptr(col_idx),
+        col_idx.numel(), int(mode), _ptr(kbar), _ptr(vsum), _ptr(Hbar), _ptr(O),
+        _ptr(workspace), ws_bytes, int(wait_ns), _ptr(status), _stream(stream)),
+        "bsa_selftest_forward_timeout")
 
 
 # ------------------------------------------------------------ allocating helpers

@@ -29,6 +29,10 @@ bsa_status check_shape(const Shape& s) {
 
 bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
+bool workspace_ok(size_t need, const void* ws, size_t ws_bytes) {
+  return need == 0 || (ws != nullptr && ws_bytes >= need && aligned16(ws));
+}
+
 int mask_blocks(const bsa_mask_desc* d) {
   if (d == nullptr) return -1;
   if (d->n_text_blocks < 0 || d->grid_h < 0 || d->grid_w < 0 || d->radius < 0 ||
@@ -41,6 +45,55 @@ int mask_blocks(const bsa_mask_desc* d) {
 }
 
 }  // namespace
+
+namespace bsa {
+
+float forward_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / sqrtf((float)d); }
+
+ForwardArgs forward_args(const void* Q, const void* K, const void* V, int Bt, int H, int L, int d,
+                         int block, const int32_t* key_valid, const int32_t* row_ptr,
+                         const int32_t* col_idx, int64_t nnz_total, int csr_per_head, int mode,
+                         const float* kbar, const float* vsum, const float* Hbar, float scale,
+                         void* O, float* lse, void* ws, int32_t* status) {
+  ForwardArgs a;
+  a.s = Shape{Bt, H, L, d, block, key_valid};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.nnz_total = nnz_total;
+  a.csr_per_head = csr_per_head;
+  a.mode = mode;
+  a.kbar = kbar;
+  a.vsum = vsum;
+  a.Hbar = Hbar;
+  a.scale = scale;
+  a.O = O;
+  a.lse = lse;
+  a.ws = ws;
+  a.status = status;
+  return a;
+}
+
+bsa_status check_forward_args(const ForwardArgs& a) {
+  bsa_status r = check_shape(a.s);
+  if (r != BSA_OK) return r;
+  if (!a.Q || !a.K || !a.V || !a.O || !a.row_ptr) return BSA_ERR_INVALID_ARG;
+  if (a.nnz_total < 0 || (a.nnz_total > 0 && a.col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
+  if (a.nnz_total >= INT32_MAX) return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(a.Q) || !aligned16(a.K) || !aligned16(a.V) || !aligned16(a.O))
+    return BSA_ERR_INVALID_ARG;
+  if (a.csr_per_head != 0 && a.csr_per_head != 1) return BSA_ERR_INVALID_ARG;
+  if (a.mode != BSA_MODE_KEEP_OR_DROP && a.mode != BSA_MODE_PISA &&
+      a.mode != BSA_MODE_PISA_BLOCK)
+    return BSA_ERR_INVALID_ARG;
+  if (a.mode == BSA_MODE_PISA && (!a.kbar || !a.vsum || !a.Hbar)) return BSA_ERR_INVALID_ARG;
+  if (!(a.scale >= 0.f)) return BSA_ERR_INVALID_ARG;
+  return BSA_OK;
+}
+
+}  // namespace bsa
 
 extern "C" {
 
@@ -92,9 +145,7 @@ bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int32_t H, i
   if (r != BSA_OK) return r;
   if (!K || !V || !kbar || !vsum || !Hbar || !Mnorm) return BSA_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V)) return BSA_ERR_INVALID_ARG;
-  const size_t need = bsa::precompute_workspace(s);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
-    return BSA_ERR_WORKSPACE;
+  if (!workspace_ok(bsa::precompute_workspace(s), workspace, ws_bytes)) return BSA_ERR_WORKSPACE;
   return from_cuda(bsa::launch_precompute(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, workspace,
                                           status, static_cast<cudaStream_t>(stream)));
 }
@@ -111,7 +162,7 @@ bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32
   if (k_top < 1 || k_top > s.M()) return BSA_ERR_INVALID_ARG;
   if ((int64_t)s.BH() * s.M() * k_top >= INT32_MAX) return BSA_ERR_UNSUPPORTED;
   if (!(lambda >= 0.f) || !(scale >= 0.f)) return BSA_ERR_INVALID_ARG;
-  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  const float sc = bsa::forward_scale(scale, d);
   return from_cuda(bsa::launch_route(s, Q, kbar, Mnorm, k_top, lambda, sc, row_ptr, col_idx,
                                      scores, status, static_cast<cudaStream_t>(stream)));
 }
@@ -123,40 +174,30 @@ bsa_status bsa_forward(const void* Q, const void* K, const void* V, int32_t Bt, 
                        int32_t mode, const float* kbar, const float* vsum,
                        const float* Hbar, float scale, void* O, float* lse,
                        void* workspace, size_t ws_bytes, int32_t* status, void* stream) {
-  const Shape s{Bt, H, L, d, block, key_valid};
-  bsa_status r = check_shape(s);
+  const bsa::ForwardArgs a = bsa::forward_args(Q, K, V, Bt, H, L, d, block, key_valid, row_ptr,
+                                               col_idx, nnz_total, csr_per_head, mode, kbar,
+                                               vsum, Hbar, scale, O, lse, workspace, status);
+  const bsa_status r = bsa::check_forward_args(a);
   if (r != BSA_OK) return r;
-  if (!Q || !K || !V || !O || !row_ptr) return BSA_ERR_INVALID_ARG;
-  if (nnz_total < 0 || (nnz_total > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
-  if (nnz_total >= INT32_MAX) return BSA_ERR_UNSUPPORTED;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
-    return BSA_ERR_INVALID_ARG;
-  if (csr_per_head != 0 && csr_per_head != 1) return BSA_ERR_INVALID_ARG;
-  if (mode != BSA_MODE_KEEP_OR_DROP && mode != BSA_MODE_PISA && mode != BSA_MODE_PISA_BLOCK)
-    return BSA_ERR_INVALID_ARG;
-  if (mode == BSA_MODE_PISA && (!kbar || !vsum || !Hbar)) return BSA_ERR_INVALID_ARG;
-  if (!(scale >= 0.f)) return BSA_ERR_INVALID_ARG;
-  const size_t need = bsa::forward_workspace(s);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
-    return BSA_ERR_WORKSPACE;
-  bsa::ForwardArgs a;
-  a.s = s;
-  a.Q = Q;
-  a.K = K;
-  a.V = V;
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.nnz_total = nnz_total;
-  a.csr_per_head = csr_per_head;
-  a.mode = mode;
-  a.kbar = kbar;
-  a.vsum = vsum;
-  a.Hbar = Hbar;
-  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
-  a.O = O;
-  a.lse = lse;
-  a.ws = workspace;
-  a.status = status;
+  if (!workspace_ok(bsa::forward_workspace(a.s), workspace, ws_bytes)) return BSA_ERR_WORKSPACE;
+  return from_cuda(bsa::launch_forward(a, static_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_selftest_forward_timeout(const void* Q, const void* K, const void* V, int32_t Bt,
+                                        int32_t H, int32_t L, int32_t d, int32_t block,
+                                        const int32_t* row_ptr, const int32_t* col_idx,
+                                        int64_t nnz_total, int32_t mode, const float* kbar,
+                                        const float* vsum, const float* Hbar, void* O,
+                                        void* workspace, size_t ws_bytes, int64_t wait_ns,
+                                        int32_t* status, void* stream) {
+  if (status == nullptr || wait_ns < 1 || wait_ns > 10000000000ll) return BSA_ERR_INVALID_ARG;
+  bsa::ForwardArgs a = bsa::forward_args(Q, K, V, Bt, H, L, d, block, nullptr, row_ptr, col_idx,
+                                         nnz_total, 1, mode, kbar, vsum, Hbar, 0.f, O, nullptr,
+                                         workspace, status);
+  const bsa_status r = bsa::check_forward_args(a);
+  if (r != BSA_OK) return r;
+  if (!workspace_ok(bsa::forward_workspace(a.s), workspace, ws_bytes)) return BSA_ERR_WORKSPACE;
+  a.wait_ns = static_cast<uint64_t>(wait_ns);
   return from_cuda(bsa::launch_forward(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -72,7 +72,9 @@ __global__ void k_validate_csr(const int32_t* __restrict__ row_ptr,
 
 size_t forward_workspace(const Shape& s) { return forward_tc_workspace(s); }
 
-cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t st) {
+cudaError_t launch_forward(const ForwardArgs& args, cudaStream_t st) {
+  ForwardArgs a = args;
+  a.scale = forward_scale(args.scale, args.s.d);
   const Shape& s = a.s;
   const int M = s.M();
   int32_t* flag = static_cast<int32_t*>(a.ws);

@@ -85,6 +85,7 @@ struct Params {
   float* lse;
   const int32_t* flag;
   int32_t* status;
+  uint64_t wait_ns;  // limit of every bounded wait
 };
 
 template <int D, int BKV>
@@ -334,7 +335,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       auto load = [&](int kind, int j, int bh) -> bool {
         const int slot = ring % C::NSLOT;
         const uint32_t ph = (ring / C::NSLOT) & 1;
-        if (!mbar_wait(&bars.kv_empty[slot], ph ^ 1, abort_flag)) return false;
+        if (!mbar_wait(&bars.kv_empty[slot], ph ^ 1, abort_flag, p.wait_ns)) return false;
         unsigned char* dst = sSlot + slot * C::SLOT;
         const CUtensorMap* map;
         int y, rows;
@@ -405,7 +406,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       constexpr uint32_t idesc_s_ch = idesc_bf16_f32(kBQ, kChunk, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, D, false, true);
       auto wait_slot = [&](uint32_t& addr) -> bool {
-        if (!mbar_wait(&bars.kv_full[slot], phase, abort_flag)) return false;
+        if (!mbar_wait(&bars.kv_full[slot], phase, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         addr = smem_u32(sSlot + slot * C::SLOT);
         last = slot;
@@ -437,8 +438,9 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (s.t == 0) {
           // item start: its Q is loaded and the previous item's epilogue has read
           // this stream's S (first-order T) and O
-          if (!mbar_wait(&bars.q_full[x], s.items & 1, abort_flag)) return false;
-          if (s.items > 0 && !mbar_wait(&bars.o_free[x], (s.items - 1) & 1, abort_flag))
+          if (!mbar_wait(&bars.q_full[x], s.items & 1, abort_flag, p.wait_ns)) return false;
+          if (s.items > 0 &&
+              !mbar_wait(&bars.o_free[x], (s.items - 1) & 1, abort_flag, p.wait_ns))
             return false;
           tc_fence_after();
           if (s.n == 0) {
@@ -463,7 +465,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const uint32_t v_slot = last;
         const bool more = s.t < s.n;
         if (more && !wait_slot(k_addr)) return false;
-        if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         {
           const int kdim = u >= s.n_ex ? kChunk : BKV;
@@ -630,7 +632,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
           }
         }
-        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag);
+        ok = mbar_wait(&bars.s_full[x], (tiles + t) & 1, abort_flag, p.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
@@ -716,7 +718,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
       if (!ok) break;
 
       // ---------------------------------------------------------------- epilogue
-      ok = mbar_wait(&bars.o_final[x], k & 1, abort_flag);
+      ok = mbar_wait(&bars.o_final[x], k & 1, abort_flag, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -774,7 +776,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         mbar_arrive(&bars.o_staged[x]);  // this row is staged
         bool staged = true;
         if (q_loader) {
-          staged = mbar_wait(&bars.o_staged[x], k & 1, abort_flag);
+          staged = mbar_wait(&bars.o_staged[x], k & 1, abort_flag, p.wait_ns);
           if (staged) {
             tma_store_4d(&tmO, sq, 0, qt * kBQ, 0, bh);  // rows past L are not written
             bulk_commit_group();
@@ -929,6 +931,7 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.lse = a.lse;
   p.flag = flag;
   p.status = a.status;
+  p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitTimeoutNs;
   cudaError_t e = cudaFuncSetAttribute(k_forward<D, BKV, kLinear>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

@@ -44,7 +44,22 @@ struct ForwardArgs {
   float* lse;
   void* ws;
   int32_t* status;
+  uint64_t wait_ns = 0;  // limit of the attention kernel's bounded waits; 0: the default
 };
+
+// bsa_forward's arguments as one record (the scale as given; 0 is resolved at launch).
+ForwardArgs forward_args(const void* Q, const void* K, const void* V, int Bt, int H, int L, int d,
+                         int block, const int32_t* key_valid, const int32_t* row_ptr,
+                         const int32_t* col_idx, int64_t nnz_total, int csr_per_head, int mode,
+                         const float* kbar, const float* vsum, const float* Hbar, float scale,
+                         void* O, float* lse, void* ws, int32_t* status);
+
+// Host-side checks of bsa_forward's arguments, all but the workspace: shapes, pointers,
+// alignment, list sizes, mode, scale. BSA_OK or the status to return.
+bsa_status check_forward_args(const ForwardArgs& a);
+
+// The scale a forward call uses: `scale`, or 1/sqrt(d) when it is 0.
+float forward_scale(float scale, int d);
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t st);
 

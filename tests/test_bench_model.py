@@ -54,3 +54,22 @@ def test_density_to_top_k():
     assert W["image_pisa"].top_k() == 5       # 15% of 32, rounded up
     assert W["sweep_L32768_d125_pisa"].top_k() == 32
     assert W["sweep_L4096_d1000_pisa"].top_k() == 32
+
+
+def test_l2_rule_per_workload():
+    """Inputs that fit twice in L2 (126 MB) are timed with a flush before every step;
+    the headline workload's inputs are far larger than L2."""
+    assert bench.input_bytes(W["video_pisa"]) == 3 * 40 * 16384 * 128 * 2
+    assert not bench.needs_flush(W["video_pisa"])
+    assert not bench.needs_flush(W["sweep_L32768_d125_pisa"])
+    for small in ("tiny_pisa", "multimodal_dit", "image_pisa", "sweep_L4096_d125_pisa"):
+        assert bench.needs_flush(W[small]), small
+    assert bench.config_of(W["image_pisa"], 1)["l2"].startswith("L2 flushed")
+
+
+def test_both_arms_name_the_workload_alike():
+    """The reference arm and this arm build their config from one function."""
+    for name in ("video_pisa", "multimodal_dit", "text_image_pisa"):
+        c = bench.config_of(W[name], 1)
+        assert c["workload"] == name and "l2" in c and "lists" in c
+    assert set(bench.SWEEP_WORKLOADS) <= set(W)

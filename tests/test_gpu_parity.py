@@ -380,7 +380,6 @@ def test_forward_malformed_lists_set_status_and_leave_output():
 @pytest.mark.parametrize("name,heads,qblocks", [
     ("image_pisa", [0, 13], None),
     ("video_pisa", [0, 39], [0, 1, 63, 127]),
-    ("sweep_L32768_d125_pisa", [0, 23], [0, 100, 255]),
     ("text_image_pisa", [0, 11, 23], None),
 ])
 def test_pipeline_full_size_sampled(name, heads, qblocks):
@@ -395,15 +394,18 @@ def test_pipeline_maximum_blocks():
     _pipeline_sampled(w, [0], [0, 1000, 2047])
 
 
-def _pipeline_sampled(w, heads, qblocks):
+def _pipeline_sampled(w, heads, qblocks, qkv=None):
     """precompute -> route -> forward on the GPU over the whole workload, in the launch
     configuration the benchmark uses; the oracle checks the sampled heads.
 
     The forward for the sampled heads is run on the oracle's own block lists (spliced
     into the GPU-routed lists), so the output comparison does not depend on near-tie
     routing decisions; the routing itself is compared separately with the tie rule.
-    A workload with token padding passes its real-token counts to every call."""
-    q, k, v = synth.make_qkv(w)
+    A workload with token padding passes its real-token counts to every call. The
+    forward runs in the workload's mode: PISA against ``pisa_head``, keep-or-drop (the
+    routed lists as S_i, nothing outside them) against ``keep_or_drop_head``."""
+    q, k, v = synth.make_qkv(w) if qkv is None else qkv
+    pisa = w.mode == "pisa"
     kk, M, BH = w.top_k(), w.n_blocks, w.batch * w.heads
     scale = 1 / math.sqrt(w.head_dim)
     qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
@@ -429,11 +431,16 @@ def _pipeline_sampled(w, heads, qblocks):
             assert rows_agree_up_to_ties(g[i], oci[i * kk:(i + 1) * kk], osc[i], kk,
                                          forced), (h, i)
         ci_host[h * M * kk:(h + 1) * M * kk] = oci
-        ref[h] = orc.pisa_head(qf, kf, vf, orp, oci, w.block, scale, kbar, vsum, Hbar,
-                               qblocks=qblocks, key_valid=valid)
+        if pisa:
+            ref[h] = orc.pisa_head(qf, kf, vf, orp, oci, w.block, scale, kbar, vsum, Hbar,
+                                   qblocks=qblocks, key_valid=valid)
+        else:
+            ref[h] = orc.keep_or_drop_head(qf, kf, vf, orp, oci, w.block, scale,
+                                           qblocks=qblocks, key_valid=valid)
     gci = torch.from_numpy(ci_host).to(DEV)
-    O, lse = b.forward(qd, kd, vd, w.block, rp, gci, 1, b.MODE_PISA, stats=stats,
-                       want_lse=True, status=st, key_valid=kv)
+    O, lse = b.forward(qd, kd, vd, w.block, rp, gci, 1,
+                       b.MODE_PISA if pisa else b.MODE_KEEP_OR_DROP,
+                       stats=stats if pisa else None, want_lse=True, status=st, key_valid=kv)
     torch.cuda.synchronize()
     assert st.item() == 0
     Og = O.reshape(BH, w.seq_len, w.head_dim)
@@ -443,3 +450,47 @@ def _pipeline_sampled(w, heads, qblocks):
         mx, rl = assert_close_out(Og[h, rows], ref[h][0], f"{w.name} head {h}")
         print(f"[parity] {w.name} head {h} max-abs {mx:.2e} rel-L2 {rl:.2e}")
     assert torch.isfinite(O.float()).all()
+
+
+# ------------------------------------------------ long-sequence sweep (every point)
+SWEEP = [n for n in synth.workloads() if n.startswith("sweep_L")]
+
+
+def _sweep_qblocks(M, seed):
+    """Query blocks to check: the first two, the last two (the last items of the
+    persistent schedule when the head is the last one), the quarter points and four
+    seeded others: at least 8 distinct blocks."""
+    fixed = {0, 1, M // 4, M // 2, 3 * M // 4, M - 2, M - 1}
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(M, size=min(M, 12), replace=False).tolist()
+    for x in extra:
+        if len(fixed) >= 11:
+            break
+        fixed.add(int(x))
+    return sorted(fixed)
+
+
+_SWEEP_QKV = {}
+
+
+def _sweep_inputs(w):
+    """The sweep workloads of one length share their inputs (same generator, grid and
+    seed; only the density and mode differ): generate once per length."""
+    key = (w.seq_len, w.heads, w.generator, w.grid)
+    if key not in _SWEEP_QKV:
+        _SWEEP_QKV.clear()
+        _SWEEP_QKV[key] = synth.make_qkv(w)
+    return _SWEEP_QKV[key]
+
+
+@pytest.mark.parametrize("name", sorted(SWEEP, key=lambda n: (synth.workloads()[n].seq_len, n)))
+def test_sweep_point_full_size_sampled(name):
+    """Every point of the long-sequence sweep (L 4K..32K x density 100/25/12.5% x
+    keep-or-drop / PISA, 24 heads) through the whole path at full size: routing of the
+    first and last head against the oracle (tie rule), and the forward output of at
+    least 8 query blocks of each, the first and last blocks included. The last head's
+    blocks are the last items of the persistent schedule (its final wave)."""
+    w = synth.workloads()[name]
+    assert len(SWEEP) == 24
+    BH = w.batch * w.heads
+    _pipeline_sampled(w, [0, BH - 1], _sweep_qblocks(w.n_blocks, w.seq_len), _sweep_inputs(w))

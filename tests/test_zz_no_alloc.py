@@ -7,7 +7,8 @@ the library. These tests call it through the C ABI twice in a row, with differen
 shapes and modes so that the second call starts from the first call's leftover scratch,
 and check each result against bsa_forward (which takes a caller-allocated workspace)
 within the parity tolerance. They also check that a shape needing more scratch than the
-built-in array is refused before anything is launched.
+built-in array is refused before anything is launched, and that keep-or-drop, which needs
+only a flag word of scratch, runs on a shape whose PISA scratch would not fit.
 """
 import ctypes
 import math
@@ -84,7 +85,33 @@ def test_noalloc_refuses_shapes_beyond_its_scratch(cuda_ok):
                                      b.MODE_PISA, p, p, p, 0.0, p, None, None, None)
     assert rc == b.ERR_SCRATCH_LIMIT
     assert b.status_string(rc) == "BSA_ERR_SCRATCH_LIMIT"
-    # the same shape in keep-or-drop needs only the flag word and is accepted by the
-    # size check (not launched here: the pointers are placeholders)
     need = b.bsa_workspace_bytes(b.CALL_FORWARD, 1, 256, 32768, 128, 128)
     assert need > b.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_keep_or_drop_runs_where_pisa_scratch_would_not_fit(cuda_ok):
+    """1024 heads of L = 256, d = 128: bsa_forward's workspace (the bf16 PISA statistics,
+    padded to 128 blocks per head) is about 34 MB, more than the built-in array. In
+    keep-or-drop mode bsa_forward_noalloc needs only the flag word and runs, matching
+    bsa_forward; the same call in PISA mode is refused with BSA_ERR_SCRATCH_LIMIT."""
+    Bt, H, L, d, block = 1, 1024, 256, 128, 128
+    assert b.bsa_workspace_bytes(b.CALL_FORWARD, Bt, H, L, d, block) > b.NOALLOC_SCRATCH_BYTES
+    g = torch.Generator().manual_seed(12)
+    q, k, v = (torch.randn(Bt, H, L, d, generator=g).to(torch.bfloat16).to(DEV)
+               for _ in range(3))
+    rp = torch.tensor([0, 1, 3], dtype=torch.int32, device=DEV)   # one list for every head
+    ci = torch.tensor([1, 0, 1], dtype=torch.int32, device=DEV)
+    st_ref = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ref, _ = b.forward(q, k, v, block, rp, ci, 0, b.MODE_KEEP_OR_DROP, status=st_ref)
+    O = torch.full_like(q, 3.0)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    b.bsa_forward_noalloc(q, k, v, block, rp, ci, 0, b.MODE_KEEP_OR_DROP, None, None, None,
+                          0.0, O, None, st)
+    torch.cuda.synchronize()
+    assert st_ref.item() == 0 and st.item() == 0
+    assert_close_out(O.reshape(-1, d), f64(ref).reshape(-1, d), "noalloc vs bsa_forward")
+    with pytest.raises(b.BsaError) as e:
+        f = torch.zeros(Bt * H, L // block, d, dtype=torch.float32, device=DEV)
+        h = torch.zeros(Bt * H, d, d, dtype=torch.float32, device=DEV)
+        b.bsa_forward_noalloc(q, k, v, block, rp, ci, 0, b.MODE_PISA, f, f, h, 0.0, O, None, st)
+    assert e.value.code == b.ERR_SCRATCH_LIMIT
