@@ -43,12 +43,14 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "forward_tiles.cuh"
 #include "sm100.cuh"
 
 namespace bsa {
 namespace fwdtc {
 
 using namespace sm100;
+using namespace fwdtiles;
 
 constexpr int kBQ = 128;       // query rows per tile
 constexpr int kChunk = 128;    // centroids per sweep tile
@@ -65,11 +67,6 @@ constexpr int kRegsSoftmax = 208;
 static_assert(128 * kRegsControl + 128 * kStreams * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-#ifndef BSA_POLY_OF8
-#define BSA_POLY_OF8 2
-#endif
-// pairs of exponentials, of every 8 pairs of an exact tile, computed on the FMA pipe
-constexpr int kPolyOf8 = BSA_POLY_OF8;
 
 struct Params {
   int L, M, BH, n_qt, n_items;
@@ -100,45 +97,6 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t O_COL(int x) { return 256u + D * x; }
 };
 
-// The key-block lists of the (one or two) query blocks of a tile, merged ascending.
-struct Lists {
-  const int32_t* col;
-  int p0, e0, p1, e1;
-  __device__ __forceinline__ int next() {
-    const int a = p0 < e0 ? __ldg(col + p0) : INT_MAX;
-    const int b = p1 < e1 ? __ldg(col + p1) : INT_MAX;
-    const int j = min(a, b);
-    if (j == INT_MAX) return -1;
-    if (a == j) ++p0;
-    if (b == j) ++p1;
-    return j;
-  }
-};
-
-template <int QBPT>
-__device__ __forceinline__ Lists item_lists(const Params& p, int bh, int qt) {
-  const int32_t* rp = p.csr_per_head ? p.row_ptr + (size_t)bh * (p.M + 1) : p.row_ptr;
-  const int i0 = qt * QBPT;
-  Lists r;
-  r.col = p.col_idx;
-  r.p0 = __ldg(rp + i0);
-  r.e0 = __ldg(rp + i0 + 1);
-  r.p1 = r.e1 = 0;
-  if (QBPT == 2 && i0 + 1 < p.M) {
-    r.p1 = r.e0;
-    r.e1 = __ldg(rp + i0 + 2);
-  }
-  return r;
-}
-
-template <int QBPT>
-__device__ __forceinline__ int count_exact(Lists l) {
-  if (QBPT == 1) return l.e0 - l.p0;
-  int n = 0;
-  while (l.next() >= 0) ++n;
-  return n;
-}
-
 // Work item k of stream x of this CTA (static schedule: the CTA takes items
 // blockIdx.x, blockIdx.x + G, ... and deals them to its two streams alternately).
 __device__ __forceinline__ int stream_item(int k, int x) {
@@ -159,7 +117,7 @@ struct StreamPos {
     if (item >= p.n_items) return;
     bh = item / p.n_qt;
     qt = item % p.n_qt;
-    lk = item_lists<QBPT>(p, bh, qt);
+    lk = item_lists<QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
     lv = lk;
     n_ex = p.linear ? p.M : count_exact<QBPT>(lk);
     n = n_ex + n_ch;
@@ -173,86 +131,6 @@ struct StreamPos {
     start(p, x, n_ch);
   }
 };
-
-// Row max of the first N columns held in registers: three-input max in four chains.
-template <int N>
-__device__ __forceinline__ float row_max(const uint32_t (&r)[128]) {
-  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-  for (int e = 0; e < N; e += 8) {
-    m0 = max3(m0, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-    m1 = max3(m1, __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-    m2 = max3(m2, __uint_as_float(r[e + 4]), __uint_as_float(r[e + 5]));
-    m3 = max3(m3, __uint_as_float(r[e + 6]), __uint_as_float(r[e + 7]));
-  }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-}
-
-// Sum of the first N columns held in registers (packed adds in four chains).
-template <int N>
-__device__ __forceinline__ float row_sum(const uint32_t (&r)[128]) {
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int q = 0; q < N / 2; ++q)
-    acc[q & 3] = add2(acc[q & 3], make_float2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])));
-  const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-  return a.x + a.y;
-}
-
-// Linear weights c1 * s + c0 for the first N columns in r, written to TMEM as bf16 pairs
-// (column c holds elements 2c and 2c + 1) at p_addr.
-template <int N>
-__device__ __forceinline__ void row_lin(const uint32_t (&r)[128], float c1, float c0,
-                                        uint32_t p_addr) {
-  const float2 a = make_float2(c1, c1), b = make_float2(c0, c0);
-#pragma unroll
-  for (int h = 0; h < N / 64; ++h) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int e = h * 64 + 2 * q;
-      const float2 w = fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a, b);
-      pk[q] = pack_bf16x2(w.x, w.y);
-    }
-    tmem_st32(p_addr + h * 32, pk);
-  }
-}
-
-// P for one row: 2^(s * scale_log2 - m_ref) for the first N columns in r, written to TMEM
-// as bf16 pairs (column c holds elements 2c and 2c + 1) at p_addr; returns the fp32 row
-// sum. With kMixed, kPolyOf8 of every 8 pairs are computed on the FMA pipe (ex2_poly2)
-// and the rest on the special-function unit, so that the two pipes share the work; a row
-// that may hold -inf (masked centroids) uses the special-function unit only.
-template <int N, bool kMixed>
-__device__ __forceinline__ float row_exp(const uint32_t (&r)[128], float scale_log2,
-                                         float m_ref, uint32_t p_addr) {
-  const float2 sc = make_float2(scale_log2, scale_log2);
-  const float2 nm = make_float2(-m_ref, -m_ref);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int h = 0; h < N / 64; ++h) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int e = h * 64 + 2 * q;
-      const float2 xx =
-          fma2(make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), sc, nm);
-      float2 ev;
-      if (kMixed && (q % 8) < kPolyOf8) {
-        ev = ex2_poly2(xx);
-      } else {
-        ev = make_float2(ex2(xx.x), ex2(xx.y));
-      }
-      acc[q & 3] = add2(acc[q & 3], ev);
-      pk[q] = pack_bf16x2(ev.x, ev.y);
-    }
-    tmem_st32(p_addr + h * 32, pk);
-  }
-  const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-  return a.x + a.y;
-}
 
 enum LoadKind { kLoadK = 0, kLoadV = 1, kLoadKbar = 2, kLoadVsum = 3, kLoadHbar = 4 };
 
@@ -551,7 +429,7 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     for (int k = 0; stream_item(k, x) < p.n_items && ok; ++k) {
       const int item = stream_item(k, x);
       const int bh = item / p.n_qt, qt = item % p.n_qt;
-      Lists lists = item_lists<C::QBPT>(p, bh, qt);
+      Lists lists = item_lists<C::QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
       const int n_ex = kLinear ? p.M : count_exact<C::QBPT>(lists);
       const int n = n_ex + n_ch;
       const int row_g = qt * kBQ + row;
@@ -655,9 +533,9 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
               if ((excl[e >> 5] >> (e & 31)) & 1u) r[e] = __float_as_uint(-INFINITY);
           }
           if (kLinear && lin)  // the block's centroid score: the mean of its row scores
-            mx = (BKV == 128 ? row_sum<128>(r) : row_sum<64>(r)) * (1.0f / BKV);
+            mx = (BKV == 128 ? row_sum<128, 128>(r) : row_sum<64, 128>(r)) * (1.0f / BKV);
           else
-            mx = cols == 128 ? row_max<128>(r) : row_max<64>(r);
+            mx = cols == 128 ? row_max<128, 128>(r) : row_max<64, 128>(r);
         }
         const float mean = mx;
         mx *= p.scale_log2;
@@ -696,14 +574,14 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
           // first-order weights about the centroid: alpha (1 + s (score - mean)); the
           // block adds B alpha to the denominator (its first-order part sums to zero)
           const float alpha = ex2(mx - m_ref);
-          row_lin<BKV>(r, alpha * p.scale, alpha * (1.0f - p.scale * mean), s_base);
+          row_lin<BKV, 128>(r, alpha * p.scale, alpha * (1.0f - p.scale * mean), s_base);
           rs = (float)BKV * alpha;
         } else if (chunk) {
-          rs = row_exp<128, false>(r, p.scale_log2, m_ref, s_base);
+          rs = row_exp<128, false, 128>(r, p.scale_log2, m_ref, s_base);
         } else if (masked) {  // -inf entries: the special-function unit gives exact zeros
-          rs = row_exp<BKV, false>(r, p.scale_log2, m_ref, s_base);
+          rs = row_exp<BKV, false, 128>(r, p.scale_log2, m_ref, s_base);
         } else {
-          rs = row_exp<BKV, true>(r, p.scale_log2, m_ref, s_base);
+          rs = row_exp<BKV, true, 128>(r, p.scale_log2, m_ref, s_base);
         }
         if (chunk) {
           l += (float)BKV * rs;
@@ -845,51 +723,6 @@ __global__ void k_stats_bf16(const float4* __restrict__ kbar, const float4* __re
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-
-// bf16 tensor [z][rows][cols] (cols contiguous, cols a multiple of 64) viewed as 4-D
-// (64 columns, rows, cols/64 column groups, z) so that one box of 64 x box_rows x
-// cols/64 lands in shared memory as cols/64 consecutive [box_rows x 64] sub-tiles, each
-// 128-byte swizzled: the operand layout of the MMA descriptors (sub-tile h at byte
-// offset h * box_rows * 128). With all_groups false the box holds one column group, for
-// callers that place the groups themselves (a Q tile shorter than 128 rows).
-bool make_map(CUtensorMap* m, const void* ptr, int cols, int rows, int z, int box_rows,
-              bool all_groups = true) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)z};
-  cuuint64_t strides[3] = {(cuuint64_t)cols * 2, 128, (cuuint64_t)cols * rows * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, all_groups ? (cuuint32_t)(cols / 64) : 1u, 1};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
 template <int D, int BKV, bool kLinear>
 cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, const void* vs16,
                 const void* hb16, cudaStream_t st) {
@@ -990,9 +823,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, const int32_t* flag, cudaStr
     if (s.d == 128 && s.block == 64) return fwdtc::run<128, 64, true>(a, flag, kb16, vs16, hb16, st);
     return fwdtc::run<128, 128, true>(a, flag, kb16, vs16, hb16, st);
   }
-  if (s.d == 64 && s.block == 64) return fwdtc::run<64, 64, false>(a, flag, kb16, vs16, hb16, st);
-  if (s.d == 64 && s.block == 128) return fwdtc::run<64, 128, false>(a, flag, kb16, vs16, hb16, st);
-  if (s.d == 128 && s.block == 64) return fwdtc::run<128, 64, false>(a, flag, kb16, vs16, hb16, st);
+  // head dim 64: the kernel whose row softmax is shared by a pair of threads
+  // (forward_pair.cu), which measured faster there; head dim 128: the kernel here
+  if (s.d == 64) return launch_forward_pair(a, flag, kb16, vs16, hb16, (int)Mp, st);
+  if (s.block == 64) return fwdtc::run<128, 64, false>(a, flag, kb16, vs16, hb16, st);
   return fwdtc::run<128, 128, false>(a, flag, kb16, vs16, hb16, st);
 }
 

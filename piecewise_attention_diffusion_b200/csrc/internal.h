@@ -74,4 +74,10 @@ cudaError_t launch_precompute_tc(const Shape& s, const void* K, const void* V, f
 size_t forward_tc_workspace(const Shape& s);
 cudaError_t launch_forward_tc(const ForwardArgs& a, const int32_t* flag, cudaStream_t st);
 
+// The attention kernel of the keep-or-drop and PISA modes at head dim 64
+// (forward_pair.cu): kb16, vs16 [BH, Mp, d] and hb16 [BH, d, d] are the bf16 statistics
+// (PISA only).
+cudaError_t launch_forward_pair(const ForwardArgs& a, const int32_t* flag, const void* kb16,
+                                const void* vs16, const void* hb16, int Mp, cudaStream_t st);
+
 }  // namespace bsa
