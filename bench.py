@@ -342,6 +342,7 @@ class Path:
             self.per_head = 1
         self.O = torch.empty_like(self.qd)
         self.ws_p = b.workspace(b.CALL_PRECOMPUTE, w.batch, w.heads, L, d, w.block, dev)
+        self.ws_r = b.workspace(b.CALL_ROUTE, w.batch, w.heads, L, d, w.block, dev)
         self.ws_f = b.workspace(b.CALL_FORWARD, w.batch, w.heads, L, d, w.block, dev)
         self.mode = {"pisa": b.MODE_PISA, "pisa_block": b.MODE_PISA_BLOCK}.get(
             w.mode, b.MODE_KEEP_OR_DROP)
@@ -361,7 +362,7 @@ class Path:
             ev[1].record(self.stream)
         if not w.mask:
             b.bsa_route(qx, s["kbar"], s["Mnorm"], w.block, self.k_top, LAMBDA, 0.0, self.rp,
-                        self.ci, None, st, key_valid=self.kv)
+                        self.ci, None, self.ws_r, st, key_valid=self.kv)
         if ev:
             ev[2].record(self.stream)
         b.bsa_forward(qx, kx, vx, w.block, self.rp, self.ci, self.per_head, self.mode,

@@ -168,12 +168,15 @@ BSA_API bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int3
  *   row_ptr  device int32 [BH, M + 1]: absolute offsets into col_idx; head h row i is
  *            col_idx[row_ptr[h*(M+1)+i] .. row_ptr[h*(M+1)+i+1]) = h*M*k_top + i*k_top ..;
  *   col_idx  device int32 [BH, M * k_top];
- *   scores   nullable fp32 [BH, M, M] receives score_ij.
+ *   scores   nullable fp32 [BH, M, M] receives score_ij;
+ *   workspace  device, >= bsa_workspace_bytes(BSA_CALL_ROUTE, ...) bytes (the column sums
+ *            of every 32-row segment of Q, BH * L/32 * d floats), contents scratch.
  * 1 <= k_top <= M. */
 BSA_API bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32_t Bt,
                      int32_t H, int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
                      int32_t k_top, float lambda, float scale, int32_t* row_ptr,
-                     int32_t* col_idx, float* scores, int32_t* status, void* stream);
+                     int32_t* col_idx, float* scores, void* workspace, size_t ws_bytes,
+                     int32_t* status, void* stream);
 
 /* bsa_forward — fused online-softmax attention over block lists.
  *   mode BSA_MODE_KEEP_OR_DROP ([BSA] §3.3):

@@ -56,7 +56,7 @@ _SIGS = {
     "bsa_precompute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp,
                               _vp, _vp, _sz, _vp, _vp]),
     "bsa_route": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _f32, _f32,
-                         _vp, _vp, _vp, _vp, _vp]),
+                         _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "bsa_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i64,
                            _i32, _i32, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "bsa_forward_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
@@ -181,7 +181,7 @@ def bsa_precompute(K, V, block, kbar, vsum, Hbar, Mnorm, Hblk=None, workspace=No
 
 
 def bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores=None,
-              status=None, stream=None, key_valid=None):
+              workspace=None, status=None, stream=None, key_valid=None):
     Bt, H, L, d = _bhld(Q, "Q")
     M = L // block
     _need(kbar, torch.float32, "kbar", (Bt * H, M, d))
@@ -190,10 +190,12 @@ def bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores
     _need(col_idx, torch.int32, "col_idx", (Bt * H * M * k_top,))
     if scores is not None:
         _need(scores, torch.float32, "scores", (Bt * H, M, M))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().bsa_route(_ptr(Q), _ptr(kbar), _ptr(Mnorm), Bt, H, L, d, block,
                            _key_valid(key_valid, L, block), k_top,
                            float(lam), float(scale), _ptr(row_ptr), _ptr(col_idx),
-                           _ptr(scores), _ptr(status), _stream(stream)), "bsa_route")
+                           _ptr(scores), _ptr(workspace), ws_bytes, _ptr(status),
+                           _stream(stream)), "bsa_route")
 
 
 def bsa_forward(Q, K, V, block, row_ptr, col_idx, csr_per_head, mode, kbar, vsum, Hbar, scale,
@@ -305,14 +307,16 @@ def precompute(K, V, block, want_blocks=False, status=None, ws=None, key_valid=N
 
 
 def route(Q, kbar, Mnorm, block, k_top, lam=1.0, scale=0.0, want_scores=False, status=None,
-          key_valid=None):
+          key_valid=None, ws=None):
     Bt, H, L, d = Q.shape
     BH, M = Bt * H, L // block
     row_ptr = torch.empty(BH * (M + 1), dtype=torch.int32, device=Q.device)
     col_idx = torch.empty(BH * M * k_top, dtype=torch.int32, device=Q.device)
     scores = torch.empty(BH, M, M, dtype=torch.float32, device=Q.device) if want_scores \
         else None
-    bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores, status,
+    if ws is None:
+        ws = workspace(CALL_ROUTE, Bt, H, L, d, block, Q.device)
+    bsa_route(Q, kbar, Mnorm, block, k_top, lam, scale, row_ptr, col_idx, scores, ws, status,
               key_valid=key_valid)
     return row_ptr, col_idx, scores
 

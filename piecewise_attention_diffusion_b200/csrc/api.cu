@@ -120,9 +120,10 @@ int32_t bsa_mask_blocks(const bsa_mask_desc* desc) { return mask_blocks(desc); }
 size_t bsa_workspace_bytes(int32_t call, int32_t Bt, int32_t H, int32_t L, int32_t d,
                            int32_t block) {
   const Shape s{Bt, H, L, d, block};
-  if (call == BSA_CALL_BUILD_MASK || call == BSA_CALL_ROUTE) return 0;
+  if (call == BSA_CALL_BUILD_MASK) return 0;
   if (check_shape(s) != BSA_OK) return 0;
   if (call == BSA_CALL_PRECOMPUTE) return bsa::precompute_workspace(s);
+  if (call == BSA_CALL_ROUTE) return bsa::route_workspace(s);
   if (call == BSA_CALL_FORWARD) return bsa::forward_workspace(s);
   return 0;
 }
@@ -153,7 +154,8 @@ bsa_status bsa_precompute(const void* K, const void* V, int32_t Bt, int32_t H, i
 bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32_t Bt,
                      int32_t H, int32_t L, int32_t d, int32_t block, const int32_t* key_valid,
                      int32_t k_top, float lambda, float scale, int32_t* row_ptr,
-                     int32_t* col_idx, float* scores, int32_t* status, void* stream) {
+                     int32_t* col_idx, float* scores, void* workspace, size_t ws_bytes,
+                     int32_t* status, void* stream) {
   const Shape s{Bt, H, L, d, block, key_valid};
   bsa_status r = check_shape(s);
   if (r != BSA_OK) return r;
@@ -162,9 +164,11 @@ bsa_status bsa_route(const void* Q, const float* kbar, const float* Mnorm, int32
   if (k_top < 1 || k_top > s.M()) return BSA_ERR_INVALID_ARG;
   if ((int64_t)s.BH() * s.M() * k_top >= INT32_MAX) return BSA_ERR_UNSUPPORTED;
   if (!(lambda >= 0.f) || !(scale >= 0.f)) return BSA_ERR_INVALID_ARG;
+  if (!workspace_ok(bsa::route_workspace(s), workspace, ws_bytes)) return BSA_ERR_WORKSPACE;
   const float sc = bsa::forward_scale(scale, d);
   return from_cuda(bsa::launch_route(s, Q, kbar, Mnorm, k_top, lambda, sc, row_ptr, col_idx,
-                                     scores, status, static_cast<cudaStream_t>(stream)));
+                                     scores, workspace, status,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_forward(const void* Q, const void* K, const void* V, int32_t Bt, int32_t H,

@@ -26,9 +26,12 @@ cudaError_t launch_precompute(const Shape& s, const void* K, const void* V, floa
                               float* vsum, float* Hbar, float* Mnorm, float* Hblk,
                               void* ws, int32_t* status, cudaStream_t st);
 
+// Routing workspace: the column sums of every 32-row segment of Q (fp32 [BH, L/32, d]).
+size_t route_workspace(const Shape& s);
+
 cudaError_t launch_route(const Shape& s, const void* Q, const float* kbar,
                          const float* Mnorm, int k_top, float lambda, float scale,
-                         int32_t* row_ptr, int32_t* col_idx, float* scores,
+                         int32_t* row_ptr, int32_t* col_idx, float* scores, void* ws,
                          int32_t* status, cudaStream_t st);
 
 struct ForwardArgs {

@@ -8,23 +8,31 @@
 //     score_ij = softmax_j(s * qbar_i . kbar_j) + lambda * M_j / sum_j' M_j'
 // (two distributions, so the mix is scale-free), qbar_i the mean query of block i.
 //
-// One CTA per (head, 8 query blocks), one warp per query block:
-//   1. pooled query: the warp streams its block of Q with 16-byte loads (the only HBM
-//      stream of the call) and reduces the columns;
-//   2. scores: thread t takes centroid j = t (looping when M > 256; with M <= 128 two
-//      threads share a centroid, half of d each, and add across the pair), reads its row
-//      once per CTA (16-byte loads from L2) and dots it with the CTA's 8 pooled queries,
-//      which every thread reads from the same shared-memory words (broadcast);
-//   3. softmax over the M blocks plus the normalised covariance term;
-//   4. exact top-k: the k-th largest score is found by a radix select on the float bit
-//      patterns (scores are >= 0, so the bit patterns order like the values), ties at
-//      the threshold go to the smaller block index, and the selected indices are
-//      compacted in ascending order with ordered ballots.
+// Two kernels:
+//   k_pool   streams Q once (the only large read of the call): one warp sums a segment
+//            of 32 rows with 16-byte loads, all of them in flight at once, and writes the
+//            column sums to the workspace (one slot per segment; no atomics, so the sums
+//            are the same bits on every run). Segments are dealt to a grid of a few CTAs
+//            per SM in a loop, so no SM is left with a partial last wave of long work;
+//   k_route  one CTA per (head, 8 query blocks), one warp per query block:
+//     1. pooled query: the sum of the block's segment sums (workspace, L2) over its
+//        number of real rows;
+//     2. scores: eight lanes share a centroid row, so that every load of kbar (from L2)
+//        reads whole 128-byte segments, and dot it with the CTA's 8 pooled queries in
+//        shared memory; a butterfly over the eight lanes adds the partial dots;
+//     3. softmax over the M blocks plus the normalised covariance term;
+//     4. exact top-k: the k-th largest score is found by a radix select on the float bit
+//        patterns (scores are >= 0, so the bit patterns order like the values), bit by
+//        bit, with the keys in registers when M <= 256; ties at the threshold go to the
+//        smaller block index, and the selected indices are compacted in ascending order
+//        with ordered ballots.
 // Token padding: the pooled query of a block averages its real rows only, and every
 // padded block (fewer than B real tokens) is forced into every list. It takes the key
 // +inf in the selection (scores are finite), so the radix select, the tie rule and the
 // compaction treat it as the largest score without a separate pass; the scores
 // written out keep the real values.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,11 +41,133 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
+constexpr int kSeg = 32;                      // rows per pooling segment
 constexpr uint32_t kForcedKey = 0x7F800000u;  // bit pattern of +inf
 
+// Column sums of every 32-row segment of Q over its real rows: partial[bh][seg][D].
 template <int B, int D>
 __global__ void __launch_bounds__(kThreads)
-k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
+k_pool(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ key_valid, int L,
+       int n_seg_total, float* __restrict__ partial, int32_t* status) {
+  constexpr int CPR = D / 8;          // 16-byte chunks per row
+  constexpr int RPI = 32 / CPR;       // rows per warp iteration
+  constexpr int NIT = kSeg / RPI;     // iterations per segment (all loads in flight)
+  const int lane = threadIdx.x % 32;
+  const int cc = lane % CPR, r0 = lane / CPR;
+  const int segs_per_head = L / kSeg;
+  const int warps = gridDim.x * kWarps;
+  for (int sg = blockIdx.x * kWarps + threadIdx.x / 32; sg < n_seg_total; sg += warps) {
+    const int bh = sg / segs_per_head, s = sg % segs_per_head;
+    const int row0 = s * kSeg;          // first row of the segment within the head
+    int nq = kSeg;                      // real rows of the segment
+    if (key_valid != nullptr) {
+      const int blk = row0 / B;
+      const int raw = __ldg(key_valid + blk);
+      if ((raw < 1 || raw > B) && lane == 0 && row0 % B == 0) report(status, BSA_ERR_BAD_PADDING);
+      const int v = min(max(raw, 1), B);
+      nq = min(kSeg, max(0, v - (row0 - blk * B)));
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(Q + ((size_t)bh * L + row0) * D) + cc;
+    uint4 u[NIT];
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) u[it] = __ldg(src + (size_t)(it * RPI + r0) * CPR);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      if (it * RPI + r0 < nq) {
+        float f[8];
+        bf16x8_to_f32(u[it], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+      }
+    }
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (lane < CPR) {
+      float4* dst = reinterpret_cast<float4*>(partial + (size_t)sg * D + cc * 8);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
+// Scores of the CTA's kWarps pooled queries (s_q, kWarps x D) against the head's M
+// centroids kb (M x D): s_sc[w][j] = scale * s_q[w] . kb[j]. Eight lanes share one
+// centroid row: lane g of the group takes the 16-byte chunks g, g + 8, g + 16, ... of the
+// row, so each load instruction of a warp reads four rows in whole 128-byte segments; the
+// eight partial dots are added across the group by a butterfly, after which lane g holds
+// query w = g's score.
+template <int D>
+__device__ __forceinline__ void score_block(const float* __restrict__ kb, bool vec, int M,
+                                            float scale, const float* s_q, float* s_sc,
+                                            int warp, int lane) {
+  constexpr int kG = 8;                 // lanes per centroid
+  constexpr int kRows = 32 / kG;        // centroids per warp pass
+  constexpr int kIt = D / (4 * kG);     // 16-byte chunks per lane per row
+  static_assert(kWarps == kG, "lane g of a group writes query block g");
+  const int g = lane % kG, rsub = lane / kG;
+  for (int j0 = warp * kRows; j0 < M; j0 += kWarps * kRows) {
+    const int j = j0 + rsub;
+    const bool valid = j < M;
+    const float* kr = kb + (size_t)(valid ? j : 0) * D;
+    float4 kv[kIt];
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      const int c = (it * kG + g) * 4;
+      kv[it] = vec ? __ldg(reinterpret_cast<const float4*>(kr + c))
+                   : make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2),
+                                 __ldg(kr + c + 3));
+    }
+    float acc[kWarps];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) acc[w] = 0.f;
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      const int c = (it * kG + g) * 4;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float4 qv = *reinterpret_cast<const float4*>(s_q + w * D + c);
+        acc[w] = fmaf(qv.w, kv[it].w,
+                      fmaf(qv.z, kv[it].z, fmaf(qv.y, kv[it].y, fmaf(qv.x, kv[it].x, acc[w]))));
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < kG; o <<= 1)
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) acc[w] += __shfl_xor_sync(0xffffffffu, acc[w], o);
+    float mine = acc[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w)
+      if (g == w) mine = acc[w];
+    if (valid) s_sc[g * M + j] = scale * mine;
+  }
+}
+
+// The k-th largest of NK * 32 keys held in registers (key j = lane + 32 q; keys of absent
+// j are 0) by a bitwise radix select: from the top bit down, T keeps a bit when at least
+// k keys are >= T with it set. Bit 31 is the sign, 0 for every key. Every candidate has a
+// bit set, so keys of 0 are never counted.
+template <int NK>
+__device__ __forceinline__ uint32_t select_kth(const uint32_t (&key)[NK], int k_top) {
+  uint32_t T = 0;
+  for (int bit = 30; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int cnt = 0;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) cnt += key[q] >= cand ? 1 : 0;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= k_top) T = cand;
+  }
+  return T;
+}
+
+// NK > 0: M <= 32 NK, and each lane keeps its scores (j = lane + 32 q) in registers from
+// the softmax to the compaction. NK == 0: any M, scores in shared memory.
+template <int B, int D, int NK>
+__global__ void __launch_bounds__(kThreads)
+k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
         const float* __restrict__ Mnorm, const int32_t* __restrict__ key_valid, int L,
         int k_top, float lambda, float scale, int32_t* __restrict__ row_ptr,
         int32_t* __restrict__ col_idx, float* __restrict__ scores, int32_t* status) {
@@ -53,12 +183,33 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   float* s_sc = s_cov + M;                      // kWarps x M
   float* s_red = s_sc + kWarps * M;             // kWarps
 
-  // normalised covariance term, shared by every query block of the head
+  // 1. the loads of the covariance terms and of the block's segment sums, all issued
+  //    before any is used
   const float* mn = Mnorm + (size_t)bh * M;
-  float part = 0.f;
-  for (int j = threadIdx.x; j < M; j += kThreads) part += __ldg(mn + j);
-  part = warp_sum(part);
-  if (lane == 0) s_red[warp] = part;
+  float mpart = 0.f;
+  for (int j = threadIdx.x; j < M; j += kThreads) mpart += __ldg(mn + j);
+  constexpr int kSegs = B / kSeg;
+  const float* ps = partial + ((size_t)bh * (L / kSeg) + (size_t)(active ? i : 0) * kSegs) * D;
+  float qs[D / 32];
+#pragma unroll
+  for (int t = 0; t < D / 32; ++t) {
+    float sum = 0.f;
+#pragma unroll
+    for (int s = 0; s < kSegs; ++s) sum += __ldg(ps + s * D + t * 32 + lane);
+    qs[t] = sum;
+  }
+  int nq = B;  // real rows of block i
+  if (key_valid != nullptr && active) nq = min(max(__ldg(key_valid + i), 1), B);
+
+  // normalised covariance term, shared by every query block of the head
+  mpart = warp_sum(mpart);
+  if (lane == 0) s_red[warp] = mpart;
+  // pooled query of block i: the mean of its real rows (zero for an idle warp, which
+  // keeps the dots below finite)
+  const float inv = active ? 1.0f / (float)nq : 0.f;
+  float* qbar = s_q + warp * D;
+#pragma unroll
+  for (int t = 0; t < D / 32; ++t) qbar[t * 32 + lane] = active ? qs[t] * inv : 0.f;
   __syncthreads();
   float msum = 0.f;
 #pragma unroll
@@ -66,166 +217,131 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   const float cov = msum > 0.f ? lambda / msum : 0.f;
   for (int j = threadIdx.x; j < M; j += kThreads) s_cov[j] = cov * __ldg(mn + j);
 
-  // 1. pooled query of block i: lanes 0..CPR-1 take row r, the next CPR lanes row r+1...
-  constexpr int CPR = D / 8;          // 16-byte chunks per row
-  constexpr int RPI = 32 / CPR;       // rows per warp iteration
-  constexpr int kUnrollQ = B / RPI >= 32 ? 16 : 8;  // loads in flight per lane
-  float* qbar = s_q + warp * D;
-  if (active) {
-    const __nv_bfloat16* qb = Q + ((size_t)bh * L + (size_t)i * B) * D;
-    const int cc = lane % CPR, r0 = lane / CPR;
-    int nq = B;  // real query rows of block i
-    if (key_valid != nullptr) {
-      const int raw = __ldg(key_valid + i);
-      if ((raw < 1 || raw > B) && lane == 0) report(status, BSA_ERR_BAD_PADDING);
-      nq = min(max(raw, 1), B);
-    }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll kUnrollQ
-    for (int r = r0; r < B; r += RPI) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(qb + (size_t)r * D) + cc);
-      float f[8];
-      bf16x8_to_f32(u, f);
-      if (r < nq) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += f[e];
-      }
-    }
-#pragma unroll
-    for (int o = CPR; o < 32; o <<= 1)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-    if (lane < CPR) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) qbar[cc * 8 + e] = acc[e] / (float)nq;
-    }
-  }
-  __syncwarp();
-
-  // 2. block scores a_j = scale * qbar_w . kbar_j for the CTA's query blocks
-  const float* kb = kbar + (size_t)bh * M * D;
-  float* sc = s_sc + warp * M;
-  if (!active) {
-#pragma unroll 1
-    for (int c = lane; c < D; c += 32) qbar[c] = 0.f;  // keep the dots below finite
-  }
-  __syncthreads();
-  // 16-byte loads when the caller's kbar allows them (each head's slice then does too,
-  // since M * D * 4 is a multiple of 16)
+  // 2. block scores a_j = scale * qbar_w . kbar_j for the CTA's query blocks. 16-byte
+  //    loads when the caller's kbar allows them (each head's slice then does too, since
+  //    M * D * 4 is a multiple of 16)
   const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
-  // with at most kThreads / 2 centroids two threads share one (half of d each)
-  const int split = 2 * M <= kThreads ? 2 : 1;
-  const int total = M * split;
-  for (int base = warp * 32; base < total; base += kThreads) {
-    const int jj = base + lane;
-    const bool valid = jj < total;
-    const int j = valid ? jj / split : 0, part = jj % split;
-    float acc[kWarps];
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) acc[w] = 0.f;
-    const float* kr = kb + (size_t)j * D;
-    const int cb = part * (D / split), ce = cb + D / split;
-#pragma unroll 4
-    for (int c = cb; c < ce; c += 4) {
-      float4 kv;
-      if (vec) {
-        kv = __ldg(reinterpret_cast<const float4*>(kr + c));
-      } else {
-        kv = make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2), __ldg(kr + c + 3));
-      }
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float4 qv = *reinterpret_cast<const float4*>(s_q + w * D + c);
-        acc[w] = fmaf(qv.w, kv.w, fmaf(qv.z, kv.z, fmaf(qv.y, kv.y, fmaf(qv.x, kv.x, acc[w]))));
-      }
-    }
-    if (split == 2) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) acc[w] += __shfl_xor_sync(0xffffffffu, acc[w], 1);
-    }
-    if (valid && part == 0) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) s_sc[w * M + j] = scale * acc[w];
-    }
-  }
+  score_block<D>(kbar + (size_t)bh * M * D, vec, M, scale, s_q, s_sc, warp, lane);
   __syncthreads();
-  __syncwarp();
   if (!active) return;
 
-  // 3. softmax over the M blocks plus the covariance term
-  float mx = -INFINITY;
-  for (int j = lane; j < M; j += 32) mx = fmaxf(mx, sc[j]);
-  mx = warp_max(mx);
-  float se = 0.f;
-  for (int j = lane; j < M; j += 32) se += expf(sc[j] - mx);
-  se = warp_sum(se);
-  const float inv_se = 1.0f / se;
+  // 3. softmax over the M blocks plus the covariance term; padded blocks take the key +inf
+  const float* sc = s_sc + warp * M;
   float* srow = scores ? scores + ((size_t)bh * M + i) * M : nullptr;
-  int n_forced = 0;
-  for (int j = lane; j < M; j += 32) {
-    const float v = expf(sc[j] - mx) * inv_se + s_cov[j];
-    const bool forced = key_valid != nullptr && __ldg(key_valid + j) < B;
-    n_forced += forced ? 1 : 0;
-    sc[j] = forced ? __uint_as_float(kForcedKey) : v;
-    if (srow) srow[j] = v;
-  }
-  n_forced = __reduce_add_sync(0xffffffffu, n_forced);
-  if (n_forced > k_top) {
-    // the list cannot hold every padded block: report, and emit a valid list anyway
-    if (lane == 0) report(status, BSA_ERR_BAD_PADDING);
-    for (int j = lane; j < M; j += 32)
-      if (__float_as_uint(sc[j]) == kForcedKey) sc[j] = 0.f;
-  }
-  __syncwarp();
-
-  // 4. k-th largest key (bit pattern of a non-negative float) by radix select
-  uint32_t T = 0;
-  if (M <= 128) {
-    // up to 4 keys per lane, held in registers for the 32 passes (absent keys 0: never
-    // counted, every candidate has a bit set)
-    uint32_t key[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = lane + 32 * q;
-      key[q] = j < M ? __float_as_uint(sc[j]) : 0u;
-    }
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      int cnt = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) cnt += key[q] >= cand ? 1 : 0;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= k_top) T = cand;
-    }
-  } else {
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      int cnt = 0;
-      for (int j = lane; j < M; j += 32) cnt += __float_as_uint(sc[j]) >= cand ? 1 : 0;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= k_top) T = cand;
-    }
-  }
-  int greater = 0;
-  for (int j = lane; j < M; j += 32) greater += __float_as_uint(sc[j]) > T ? 1 : 0;
-  greater = __reduce_add_sync(0xffffffffu, greater);
-  const int ties_needed = k_top - greater;  // >= 1
-
-  // 5. ascending compaction: selected = key > T, or key == T among the first
-  //    ties_needed such keys in index order
   const int64_t base = (int64_t)bh * M * k_top + (int64_t)i * k_top;
   const unsigned lt = (1u << lane) - 1u;
-  int ties_seen = 0, out = 0;
-  for (int j0 = 0; j0 < M; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < M ? __float_as_uint(sc[j]) : 0u;
-    const bool tie = j < M && key == T;
-    const unsigned tb = __ballot_sync(0xffffffffu, tie);
-    const bool sel = j < M && (key > T || (tie && ties_seen + __popc(tb & lt) < ties_needed));
-    const unsigned sb = __ballot_sync(0xffffffffu, sel);
-    if (sel) col_idx[base + out + __popc(sb & lt)] = j;
-    ties_seen += __popc(tb);
-    out += __popc(sb);
+  if constexpr (NK > 0) {
+    float x[NK];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) {
+      const int j = lane + 32 * q;
+      x[q] = j < M ? sc[j] : -INFINITY;
+      mx = fmaxf(mx, x[q]);
+    }
+    mx = warp_max(mx);
+    float se = 0.f;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) {
+      x[q] = lane + 32 * q < M ? expf(x[q] - mx) : 0.f;
+      se += x[q];
+    }
+    se = warp_sum(se);
+    const float inv_se = 1.0f / se;
+    uint32_t key[NK];
+    int n_forced = 0;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) {
+      const int j = lane + 32 * q;
+      key[q] = 0u;
+      if (j < M) {
+        const float v = x[q] * inv_se + s_cov[j];
+        const bool forced = key_valid != nullptr && __ldg(key_valid + j) < B;
+        n_forced += forced ? 1 : 0;
+        key[q] = forced ? kForcedKey : __float_as_uint(v);
+        if (srow) srow[j] = v;
+      }
+    }
+    n_forced = __reduce_add_sync(0xffffffffu, n_forced);
+    if (n_forced > k_top) {
+      // the list cannot hold every padded block: report, and emit a valid list anyway
+      if (lane == 0) report(status, BSA_ERR_BAD_PADDING);
+#pragma unroll
+      for (int q = 0; q < NK; ++q)
+        if (key[q] == kForcedKey) key[q] = 0u;
+    }
+
+    // 4. the k-th largest key, then 5. the ascending compaction: selected = key > T, or
+    //    key == T among the first ties_needed such keys in index order
+    const uint32_t T = select_kth<NK>(key, k_top);
+    int greater = 0;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) greater += key[q] > T ? 1 : 0;
+    greater = __reduce_add_sync(0xffffffffu, greater);
+    const int ties_needed = k_top - greater;  // >= 1
+    int ties_seen = 0, out = 0;
+#pragma unroll
+    for (int q = 0; q < NK; ++q) {
+      const int j = lane + 32 * q;
+      const bool tie = j < M && key[q] == T;
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      const bool sel = j < M && (key[q] > T || (tie && ties_seen + __popc(tb & lt) < ties_needed));
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) col_idx[base + out + __popc(sb & lt)] = j;
+      ties_seen += __popc(tb);
+      out += __popc(sb);
+    }
+  } else {
+    float* scw = s_sc + warp * M;
+    float mx = -INFINITY;
+    for (int j = lane; j < M; j += 32) mx = fmaxf(mx, scw[j]);
+    mx = warp_max(mx);
+    float se = 0.f;
+    for (int j = lane; j < M; j += 32) se += expf(scw[j] - mx);
+    se = warp_sum(se);
+    const float inv_se = 1.0f / se;
+    int n_forced = 0;
+    for (int j = lane; j < M; j += 32) {
+      const float v = expf(scw[j] - mx) * inv_se + s_cov[j];
+      const bool forced = key_valid != nullptr && __ldg(key_valid + j) < B;
+      n_forced += forced ? 1 : 0;
+      scw[j] = forced ? __uint_as_float(kForcedKey) : v;
+      if (srow) srow[j] = v;
+    }
+    n_forced = __reduce_add_sync(0xffffffffu, n_forced);
+    if (n_forced > k_top) {
+      if (lane == 0) report(status, BSA_ERR_BAD_PADDING);
+      for (int j = lane; j < M; j += 32)
+        if (__float_as_uint(scw[j]) == kForcedKey) scw[j] = 0.f;
+    }
+    __syncwarp();
+    // 4. k-th largest key by a bitwise radix select over shared memory: from the top bit
+    //    down, keep a bit of T when at least k keys are >= T with it set
+    uint32_t T = 0;
+    for (int bit = 30; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+      for (int j = lane; j < M; j += 32) cnt += __float_as_uint(scw[j]) >= cand ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= k_top) T = cand;
+    }
+    int greater = 0;
+    for (int j = lane; j < M; j += 32) greater += __float_as_uint(scw[j]) > T ? 1 : 0;
+    greater = __reduce_add_sync(0xffffffffu, greater);
+    const int ties_needed = k_top - greater;  // >= 1
+    // 5. ascending compaction
+    int ties_seen = 0, out = 0;
+    for (int j0 = 0; j0 < M; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < M ? __float_as_uint(scw[j]) : 0u;
+      const bool tie = j < M && key == T;
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      const bool sel = j < M && (key > T || (tie && ties_seen + __popc(tb & lt) < ties_needed));
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) col_idx[base + out + __popc(sb & lt)] = j;
+      ties_seen += __popc(tb);
+      out += __popc(sb);
+    }
   }
   if (lane == 0) {
     int32_t* rp = row_ptr + (size_t)bh * (M + 1);
@@ -234,37 +350,67 @@ k_route(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ kbar,
   }
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 template <int B, int D>
 cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* Mnorm,
                 int k_top, float lambda, float scale, int32_t* row_ptr, int32_t* col_idx,
-                float* scores, int32_t* status, cudaStream_t st) {
+                float* scores, void* ws, int32_t* status, cudaStream_t st) {
   const int M = s.M();
-  const size_t sm = ((size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(k_route<B, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  float* partial = static_cast<float*>(ws);
+  // pooling: as many CTAs as are resident at once, each warp looping over 32-row
+  // segments (one wave, no tail of late CTAs)
+  const int n_seg = s.BH() * (s.L / kSeg);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_pool<B, D>, kThreads, 0);
   if (e != cudaSuccess) return e;
-  k_route<B, D><<<dim3(ceil_div(M, kWarps), s.BH()), kThreads, sm, st>>>(
-      static_cast<const __nv_bfloat16*>(Q), kbar, Mnorm, s.key_valid, s.L, k_top, lambda, scale,
-      row_ptr, col_idx, scores, status);
+  const int pool_grid = std::min(ceil_div(n_seg, kWarps), std::max(per_sm, 1) * sm_count());
+  k_pool<B, D><<<pool_grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), s.key_valid,
+                                               s.L, n_seg, partial, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t sm = ((size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
+  const dim3 grid(ceil_div(M, kWarps), s.BH());
+  auto go = [&](auto kern) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kThreads, sm, st>>>(partial, kbar, Mnorm, s.key_valid, s.L, k_top, lambda, scale,
+                                     row_ptr, col_idx, scores, status);
+    return cudaSuccess;
+  };
+  if (M <= 128) e = go(k_route<B, D, 4>);
+  else if (M <= 256) e = go(k_route<B, D, 8>);
+  else e = go(k_route<B, D, 0>);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t route_workspace(const Shape& s) {
+  // one column sum of d floats per 32-row segment of Q
+  return (size_t)s.BH() * (s.L / kSeg) * s.d * sizeof(float);
+}
+
 cudaError_t launch_route(const Shape& s, const void* Q, const float* kbar, const float* Mnorm,
                          int k_top, float lambda, float scale, int32_t* row_ptr,
-                         int32_t* col_idx, float* scores, int32_t* status, cudaStream_t st) {
+                         int32_t* col_idx, float* scores, void* ws, int32_t* status,
+                         cudaStream_t st) {
   if (s.block == 64 && s.d == 64)
-    return run<64, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
-                        status, st);
+    return run<64, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, ws,
+                       status, st);
   if (s.block == 64 && s.d == 128)
-    return run<64, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
-                         status, st);
+    return run<64, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, ws,
+                        status, st);
   if (s.block == 128 && s.d == 64)
-    return run<128, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
-                         status, st);
-  return run<128, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores,
-                          status, st);
+    return run<128, 64>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, ws,
+                        status, st);
+  return run<128, 128>(s, Q, kbar, Mnorm, k_top, lambda, scale, row_ptr, col_idx, scores, ws,
+                       status, st);
 }
 
 }  // namespace bsa

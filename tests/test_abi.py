@@ -65,7 +65,9 @@ def test_mask_blocks_and_invalid_descriptors():
 
 
 def test_workspace_sizes():
-    assert b.bsa_workspace_bytes(b.CALL_ROUTE, 1, 40, 16384, 128, 128) == 0
+    # routing: one fp32 column sum of d per 32-row segment of Q
+    assert b.bsa_workspace_bytes(b.CALL_ROUTE, 1, 40, 16384, 128, 128) == 40 * 512 * 128 * 4
+    assert b.bsa_workspace_bytes(b.CALL_ROUTE, 8, 16, 1152, 64, 64) == 128 * 36 * 64 * 4
     assert b.bsa_workspace_bytes(b.CALL_PRECOMPUTE, 1, 40, 16384, 128, 128) > 0
     assert b.bsa_workspace_bytes(b.CALL_FORWARD, 1, 40, 16384, 128, 128) > 0
     assert b.bsa_workspace_bytes(b.CALL_FORWARD, 1, 4, 1000, 128, 128) == 0   # L % block
@@ -119,14 +121,18 @@ def test_forward_rejects_bad_arguments():
 def test_route_and_precompute_reject_bad_arguments():
     p = _fake()
     r = b.lib().bsa_route
-    assert r(p, p, p, 1, 2, 512, 64, 64, None, 0, 1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 0, 1.0, 0.0, p, p, None, p, 1 << 20, None, None) == \
         b.ERR_INVALID_ARG                                      # k_top 0
-    assert r(p, p, p, 1, 2, 512, 64, 64, None, 9, 1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 9, 1.0, 0.0, p, p, None, p, 1 << 20, None, None) == \
         b.ERR_INVALID_ARG                                      # k_top > M
-    assert r(p, p, p, 1, 2, 512, 64, 64, None, 2, -1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 2, -1.0, 0.0, p, p, None, p, 1 << 20, None, None) == \
         b.ERR_INVALID_ARG                                      # lambda < 0
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 2, 1.0, 0.0, p, p, None, p, 64, None, None) == \
+        b.ERR_WORKSPACE                                        # workspace too small
+    assert r(p, p, p, 1, 2, 512, 64, 64, None, 2, 1.0, 0.0, p, p, None, None, 0, None, None) == \
+        b.ERR_WORKSPACE                                        # no workspace
     odd = ctypes.c_void_p((1 << 20) + 2)                       # key_valid not 4-aligned
-    assert r(p, p, p, 1, 2, 512, 64, 64, odd, 2, 1.0, 0.0, p, p, None, None, None) == \
+    assert r(p, p, p, 1, 2, 512, 64, 64, odd, 2, 1.0, 0.0, p, p, None, p, 1 << 20, None, None) == \
         b.ERR_INVALID_ARG
     pc = b.lib().bsa_precompute
     assert pc(p, p, 1, 2, 512, 64, 64, None, p, p, p, p, None, None, 0, None, None) == \
