@@ -20,47 +20,67 @@
 namespace bsa {
 namespace {
 
+// One warp per row: the lanes read the row's entries 32 at a time (coalesced), each
+// entry is compared with its left neighbour (the previous chunk's last entry carried in
+// lane 0), and the PISA count of padded blocks in the row is a warp sum.
 __global__ void k_validate_csr(const int32_t* __restrict__ row_ptr,
                                const int32_t* __restrict__ col_idx, int64_t nnz_total, int M,
                                int n_heads, const int32_t* __restrict__ key_valid, int block,
                                bool pisa, int32_t* flag, int32_t* status) {
+  constexpr int kWarps = 8;
+  __shared__ int s_npad;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_rows = n_heads * M;
   // padded blocks (real tokens < block) and the range of every count
-  int n_pad = 0;
+  if (threadIdx.x == 0) s_npad = 0;
+  __syncthreads();
   if (key_valid != nullptr) {
-    for (int j = 0; j < M; ++j) {
+    int mine = 0;
+    for (int j = threadIdx.x; j < M; j += blockDim.x) {
       const int v = __ldg(key_valid + j);
-      n_pad += v < block ? 1 : 0;
-      if ((v < 1 || v > block) && blockIdx.x == 0 && threadIdx.x == 0) {
+      mine += v < block ? 1 : 0;
+      if ((v < 1 || v > block) && blockIdx.x == 0) {
         atomicOr(flag, 1);
         report(status, BSA_ERR_BAD_PADDING);
       }
     }
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if (lane == 0 && mine) atomicAdd(&s_npad, mine);
   }
-  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < n_rows; r += gridDim.x * blockDim.x) {
+  __syncthreads();
+  const int n_pad = s_npad;
+  for (int r = blockIdx.x * kWarps + warp; r < n_rows; r += gridDim.x * kWarps) {
     const int h = r / M, i = r % M;
     const int32_t* rp = row_ptr + (size_t)h * (M + 1);
-    const int64_t b = rp[i], e = rp[i + 1];
+    const int64_t b = __ldg(rp + i), e = __ldg(rp + i + 1);
     bool ok = b >= 0 && b <= e && e <= nnz_total && (e - b) <= M;
+    int prev = -1, in_row = 0;
     if (ok) {
-      int prev = -1;
-      for (int64_t p = b; p < e; ++p) {
-        const int c = col_idx[p];
-        if (c <= prev || c >= M) {
+      for (int64_t p0 = b; p0 < e; p0 += 32) {
+        const int64_t p = p0 + lane;
+        const bool has = p < e;
+        const int c = has ? __ldg(col_idx + p) : 0;
+        int left = __shfl_up_sync(0xffffffffu, c, 1);
+        if (lane == 0) left = prev;
+        if (__any_sync(0xffffffffu, has && (c <= left || c >= M))) {
           ok = false;
           break;
         }
-        prev = c;
+        const int64_t rem = e - 1 - p0;
+        const int last = rem < 31 ? (int)rem : 31;
+        prev = __shfl_sync(0xffffffffu, c, last);
+        if (pisa && n_pad > 0 && has) in_row += __ldg(key_valid + c) < block ? 1 : 0;
       }
     }
     if (!ok) {
-      atomicOr(flag, 1);
-      report(status, BSA_ERR_BAD_CSR);
+      if (lane == 0) {
+        atomicOr(flag, 1);
+        report(status, BSA_ERR_BAD_CSR);
+      }
     } else if (pisa && n_pad > 0) {
       // a padded block is always computed exactly: it must be in every list
-      int in_row = 0;
-      for (int64_t p = b; p < e; ++p) in_row += __ldg(key_valid + col_idx[p]) < block ? 1 : 0;
-      if (in_row != n_pad) {
+      in_row = __reduce_add_sync(0xffffffffu, in_row);
+      if (in_row != n_pad && lane == 0) {
         atomicOr(flag, 1);
         report(status, BSA_ERR_BAD_PADDING);
       }
@@ -82,7 +102,7 @@ cudaError_t launch_forward(const ForwardArgs& args, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int n_heads = a.csr_per_head ? s.BH() : 1;
   const int rows = n_heads * M;
-  k_validate_csr<<<ceil_div(rows, 256), 256, 0, st>>>(
+  k_validate_csr<<<ceil_div(rows, 8), 256, 0, st>>>(
       a.row_ptr, a.col_idx, a.nnz_total, M, n_heads, s.key_valid, s.block,
       a.mode == BSA_MODE_PISA || a.mode == BSA_MODE_PISA_BLOCK, flag, a.status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -104,6 +104,27 @@ def test_precompute_parity(name, heads):
     np.testing.assert_allclose(f64(out["Mnorm"]), Mn, rtol=1e-4, atol=1e-4 * Mn.max())
 
 
+def test_precompute_full_size_all_heads():
+    """The whole video shape (40 heads, K and V 671 MB): the first and last heads and two
+    neighbours in the middle against the oracle. Every CTA of the two passes takes a
+    contiguous piece of the flattened (head, block) range, so these heads' blocks are
+    split between CTAs, and their partial sums of H_j are added by the reduction."""
+    w = synth.workloads()["video_pisa"]
+    q, k, v = synth.make_qkv(w, seed=0)
+    st = _status()
+    out = b.precompute(k.to(DEV), v.to(DEV), w.block, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for h in (0, 8, 9, 39):
+        kbar, vsum, H, Hbar, Mn = orc.precompute_head(f64(k[0, h]), f64(v[0, h]), w.block)
+        np.testing.assert_allclose(f64(out["kbar"][h]), kbar, rtol=1e-5, atol=1e-5)
+        np.testing.assert_allclose(f64(out["vsum"][h]), vsum, rtol=1e-5, atol=1e-4)
+        scaleH = np.abs(H).max()
+        np.testing.assert_allclose(f64(out["Hbar"][h]), Hbar,
+                                   atol=2e-5 * scaleH * math.sqrt(w.block))
+        np.testing.assert_allclose(f64(out["Mnorm"][h]), Mn, rtol=1e-4, atol=1e-4 * Mn.max())
+
+
 # --------------------------------------------------------------------------- route
 @pytest.mark.parametrize("name,heads,lam", [("tiny_pisa", None, 1.0), ("tiny_pisa", None, 0.0),
                                             ("image_pisa", [1, 2], 1.0),
@@ -373,6 +394,35 @@ def test_forward_malformed_lists_set_status_and_leave_output():
         b.forward(q, k, v, w.block, grp, gci, 0, b.MODE_KEEP_OR_DROP, status=st, out=O)
         torch.cuda.synchronize()
         assert st.item() == b.ERR_BAD_CSR, (rp, ci)
+        assert (O == 7.0).all()
+
+
+def test_forward_list_checks_cross_the_32_entry_chunks():
+    """Rows of 64 entries: the check reads a row 32 entries at a time, so a duplicate
+    that straddles two chunks, a descent inside the second chunk and a negative index
+    must all be caught; the intact lists pass."""
+    w = synth.Workload("long_rows", 1, 1, 4096, 64, 64, "keep_or_drop", generator="iid")
+    q, k, v = (x.to(DEV) for x in synth.make_qkv(w, seed=2))
+    M = w.n_blocks
+    full = np.tile(np.arange(M, dtype=np.int32), M)
+    rp = np.arange(0, M * M + 1, M, dtype=np.int32)
+
+    def run(ci):
+        grp, gci = _csr_to_gpu(rp, ci)
+        st = _status()
+        O = torch.full_like(q, 7.0)
+        b.forward(q, k, v, w.block, grp, gci, 0, b.MODE_KEEP_OR_DROP, status=st, out=O)
+        torch.cuda.synchronize()
+        return st.item(), O
+
+    code, O = run(full)
+    assert code == 0
+    assert torch.isfinite(O.float()).all()
+    for row, pos, val in [(5, 32, 31), (7, 40, 39 - 2), (9, 0, -1), (63, 63, M)]:
+        ci = full.copy()
+        ci[row * M + pos] = val
+        code, O = run(ci)
+        assert code == b.ERR_BAD_CSR, (row, pos, val)
         assert (O == 7.0).all()
 
 
