@@ -76,6 +76,7 @@ constexpr uint32_t kAll = 0xffffffffu;
 
 struct Params {
   int L, M, BH, n_qt, n_items;
+  int tile_major;  // items ordered (tile, head) instead of (head, tile): lists shared by all heads
   int qbox;  // rows per Q box: 128, or L when L < 128
   const int32_t* row_ptr;
   const int32_t* col_idx;
@@ -89,6 +90,21 @@ struct Params {
   int32_t* status;
   uint64_t wait_ns;  // limit of every bounded wait
 };
+
+// Head and query tile of work item `item`. With one list shared by every head (a fixed
+// mask) the items go tile by tile, every head's tile qt before any head's tile qt + 1, so
+// that the first items dealt are the heads' first tiles (in the multimodal layout the
+// text rows, whose lists are the longest); with per-head lists, head by head (a head's
+// K and V stay in L2 while its tiles run).
+__device__ __forceinline__ void item_tile(const Params& p, int item, int& bh, int& qt) {
+  if (p.tile_major) {
+    qt = item / p.BH;
+    bh = item % p.BH;
+  } else {
+    bh = item / p.n_qt;
+    qt = item % p.n_qt;
+  }
+}
 
 template <int D, int BKV>
 struct Cfg {
@@ -129,8 +145,7 @@ struct StreamPos {
   __device__ __forceinline__ void start(const Params& p, int x, int n_ch) {
     item = stream_item(k, x);
     if (item >= p.n_items) return;
-    bh = item / p.n_qt;
-    qt = item % p.n_qt;
+    item_tile(p, item, bh, qt);
     lk = item_lists<QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
     lv = lk;
     n_ex = count_exact<QBPT>(lk);
@@ -163,8 +178,9 @@ __device__ __forceinline__ void tail_bits(int v, uint32_t& w0, uint32_t& w1) {
 // sums: of the stored bf16 values (x), which normalise the output, so that every output
 // is a weighted mean of value rows with the same weights in numerator and denominator;
 // and of the fp32 values (y), for the log-sum-exp. With kMixed, kPolyOf8 of every 8 pairs
-// run on the FMA pipe.
-template <int N, bool kMixed>
+// run on the FMA pipe; with kMasked (a tile with excluded columns, -inf in r) those give
+// exactly 0 for an excluded column, as the special-function unit does.
+template <int N, bool kMixed, bool kMasked>
 __device__ __forceinline__ float2 half_exp(const uint32_t (&r)[32], float scale_log2, float m_ref,
                                            uint32_t p_addr) {
   const float2 sc = make_float2(scale_log2, scale_log2);
@@ -181,6 +197,11 @@ __device__ __forceinline__ float2 half_exp(const uint32_t (&r)[32], float scale_
       float2 ev;
       if (kMixed && q < kPolyOf8) {
         ev = ex2_poly2(xx);
+        if (kMasked) {
+          // the polynomial clamps its argument at -126: a masked score (-inf) must give 0
+          ev.x = xx.x == -INFINITY ? 0.f : ev.x;
+          ev.y = xx.y == -INFINITY ? 0.f : ev.y;
+        }
       } else {
         ev = make_float2(ex2(xx.x), ex2(xx.y));
       }
@@ -474,7 +495,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
     const uint32_t o_half = tmem + lane_addr + C::O_COL(x) + hf * C::HALF_D;
     unsigned char* sq = smem + x * C::QBYTES;
     auto load_q = [&](int item) {
-      const int bh = item / p.n_qt, qt = item % p.n_qt;
+      int bh, qt;
+      item_tile(p, item, bh, qt);
       mbar_arrive_expect_tx(&bars.q_full[x], p.qbox * D * 2);
       if (p.qbox == kBQ) {
         tma_load_4d(sq, &tmQ, &bars.q_full[x], 0, qt * kBQ, 0, bh);
@@ -493,7 +515,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
     bool ok = true;
     for (int k = 0; stream_item(k, x) < p.n_items && ok; ++k) {
       const int item = stream_item(k, x);
-      const int bh = item / p.n_qt, qt = item % p.n_qt;
+      int bh, qt;
+      item_tile(p, item, bh, qt);
       Lists lists = item_lists<C::QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
       const int n_ex = count_exact<C::QBPT>(lists);
       const int n = n_ex + n_ch;
@@ -625,8 +648,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
           for (int e = 0; e < 8; ++e) z[e] = 0u;
           for (int c = 0; c < w / 2; c += 8) tmem_st8(a + c, z);
         } else {
-          rs = masked ? half_exp<32, false>(r, p.scale_log2, m_ref, a)
-                      : half_exp<32, true>(r, p.scale_log2, m_ref, a);
+          rs = masked ? half_exp<32, true, true>(r, p.scale_log2, m_ref, a)
+                      : half_exp<32, true, false>(r, p.scale_log2, m_ref, a);
           if (w == 64) {
             tmem_ld32(a + 32, r);
             tmem_wait_ld();
@@ -635,8 +658,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
               for (int e = 0; e < 32; ++e)
                 if ((ex1 >> e) & 1u) r[e] = __float_as_uint(-INFINITY);
             }
-            const float2 r2 = masked ? half_exp<32, false>(r, p.scale_log2, m_ref, a + 16)
-                                     : half_exp<32, true>(r, p.scale_log2, m_ref, a + 16);
+            const float2 r2 = masked ? half_exp<32, true, true>(r, p.scale_log2, m_ref, a + 16)
+                                     : half_exp<32, true, false>(r, p.scale_log2, m_ref, a + 16);
             rs = make_float2(rs.x + r2.x, rs.y + r2.y);
           }
         }
@@ -786,6 +809,7 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.BH = BH;
   p.n_qt = ceil_div(s.L, kBQ);
   p.n_items = BH * p.n_qt;
+  p.tile_major = a.csr_per_head ? 0 : 1;
   p.qbox = qbox;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;

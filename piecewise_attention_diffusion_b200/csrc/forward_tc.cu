@@ -70,6 +70,7 @@ constexpr float kRescaleLog2 = 8.0f;
 
 struct Params {
   int L, M, BH, n_qt, n_items;
+  int tile_major;  // items ordered (tile, head) instead of (head, tile): lists shared by all heads
   int qbox;  // rows per Q box: 128, or L when L < 128
   const int32_t* row_ptr;
   const int32_t* col_idx;
@@ -84,6 +85,21 @@ struct Params {
   int32_t* status;
   uint64_t wait_ns;  // limit of every bounded wait
 };
+
+// Head and query tile of work item `item`. With one list shared by every head (a fixed
+// mask) the items go tile by tile, every head's tile qt before any head's tile qt + 1, so
+// that the first items dealt are the heads' first tiles (in the multimodal layout the
+// text rows, whose lists are the longest); with per-head lists, head by head (a head's
+// K and V stay in L2 while its tiles run).
+__device__ __forceinline__ void item_tile(const Params& p, int item, int& bh, int& qt) {
+  if (p.tile_major) {
+    qt = item / p.BH;
+    bh = item % p.BH;
+  } else {
+    bh = item / p.n_qt;
+    qt = item % p.n_qt;
+  }
+}
 
 template <int D, int BKV>
 struct Cfg {
@@ -115,8 +131,7 @@ struct StreamPos {
   __device__ __forceinline__ void start(const Params& p, int x, int n_ch) {
     item = stream_item(k, x);
     if (item >= p.n_items) return;
-    bh = item / p.n_qt;
-    qt = item % p.n_qt;
+    item_tile(p, item, bh, qt);
     lk = item_lists<QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
     lv = lk;
     n_ex = p.linear ? p.M : count_exact<QBPT>(lk);
@@ -409,7 +424,8 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t o_base = tmem + lane_addr + C::O_COL(x);
     unsigned char* sq = smem + x * C::QBYTES;
     auto load_q = [&](int item) {
-      const int bh = item / p.n_qt, qt = item % p.n_qt;
+      int bh, qt;
+      item_tile(p, item, bh, qt);
       mbar_arrive_expect_tx(&bars.q_full[x], p.qbox * D * 2);
       if (p.qbox == kBQ) {
         tma_load_4d(sq, &tmQ, &bars.q_full[x], 0, qt * kBQ, 0, bh);
@@ -428,7 +444,8 @@ k_forward(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     bool ok = true;
     for (int k = 0; stream_item(k, x) < p.n_items && ok; ++k) {
       const int item = stream_item(k, x);
-      const int bh = item / p.n_qt, qt = item % p.n_qt;
+      int bh, qt;
+      item_tile(p, item, bh, qt);
       Lists lists = item_lists<C::QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
       const int n_ex = kLinear ? p.M : count_exact<C::QBPT>(lists);
       const int n = n_ex + n_ch;
@@ -751,6 +768,7 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.BH = BH;
   p.n_qt = ceil_div(s.L, kBQ);
   p.n_items = BH * p.n_qt;
+  p.tile_major = a.csr_per_head ? 0 : 1;
   p.qbox = qbox;
   p.row_ptr = a.row_ptr;
   p.col_idx = a.col_idx;
