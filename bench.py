@@ -471,24 +471,29 @@ def run_ours(args, w, world, rank, local):
         sets = [(qd, kd, vd, O),
                 (torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd),
                  torch.empty_like(O))]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        # one input stream per tensor, so that the three copies can run on separate copy
+        # engines at once
+        s_ins = [torch.cuda.Stream(dev) for _ in range(3)]
+        s_out = torch.cuda.Stream(dev)
 
         def e2e_steps(n, start_ev=None):
             ev = lambda: torch.cuda.Event()
-            in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+            in_done = [[ev(), ev(), ev()], [ev(), ev(), ev()]]
+            comp_done, out_done = [ev(), ev()], [ev(), ev()]
             if start_ev is not None:
-                s_in.wait_event(start_ev)
+                for s_in in s_ins:
+                    s_in.wait_event(start_ev)
             for i in range(n):
                 x = i % 2
                 qx, kx, vx, ox = sets[x]
-                with torch.cuda.stream(s_in):
-                    if i >= 2:
-                        s_in.wait_event(comp_done[x])  # step i-2 has read this set
-                    qx.copy_(qh, non_blocking=True)
-                    kx.copy_(kh, non_blocking=True)
-                    vx.copy_(vh, non_blocking=True)
-                    in_done[x].record(s_in)
-                stream.wait_event(in_done[x])
+                for s_in, dst, src, done in zip(s_ins, (qx, kx, vx), (qh, kh, vh), in_done[x]):
+                    with torch.cuda.stream(s_in):
+                        if i >= 2:
+                            s_in.wait_event(comp_done[x])  # step i-2 has read this set
+                        dst.copy_(src, non_blocking=True)
+                        done.record(s_in)
+                for done in in_done[x]:
+                    stream.wait_event(done)
                 if i >= 2:
                     stream.wait_event(out_done[x])     # step i-2's output has been read
                 path.step(qx, kx, vx, out=ox)
