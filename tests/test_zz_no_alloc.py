@@ -115,3 +115,42 @@ def test_noalloc_keep_or_drop_runs_where_pisa_scratch_would_not_fit(cuda_ok):
         h = torch.zeros(Bt * H, d, d, dtype=torch.float32, device=DEV)
         b.bsa_forward_noalloc(q, k, v, block, rp, ci, 0, b.MODE_PISA, f, f, h, 0.0, O, None, st)
     assert e.value.code == b.ERR_SCRATCH_LIMIT
+
+
+def test_noalloc_keep_or_drop_with_two_blocks_per_tile(cuda_ok):
+    """Block 64: every 128-row tile runs the merged lists of two query blocks, each row
+    masking the key blocks its own block does not select. Pairs of rows whose lists
+    overlap, nest and are disjoint, per head; bsa_forward_noalloc against bsa_forward and
+    against the oracle."""
+    Bt, H, L, d, block = 1, 2, 512, 64, 64
+    M = L // block
+    g = torch.Generator().manual_seed(13)
+    q, k, v = (torch.randn(Bt, H, L, d, generator=g).to(torch.bfloat16).to(DEV)
+               for _ in range(3))
+    lists = [[0, 1, 2], [1, 2, 3],          # overlap
+             [0, 2, 4, 6], [2, 4],          # nested
+             [0, 1], [5, 7],                # disjoint
+             [7], [0, 3, 6, 7]]
+    rows = [lists, list(reversed(lists))]   # head 1: the same lists, other pairs
+    rp, ci = [], []
+    for h in range(H):
+        base = h * sum(len(r) for r in rows[h])
+        rp.append(np.cumsum([0] + [len(r) for r in rows[h]]) + base)
+        ci.extend(c for r in rows[h] for c in sorted(r))
+    rp = torch.tensor(np.concatenate(rp), dtype=torch.int32, device=DEV)
+    ci = torch.tensor(ci, dtype=torch.int32, device=DEV)
+    st_ref = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ref, _ = b.forward(q, k, v, block, rp, ci, 1, b.MODE_KEEP_OR_DROP, status=st_ref)
+    O = torch.full_like(q, 3.0)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    b.bsa_forward_noalloc(q, k, v, block, rp, ci, 1, b.MODE_KEEP_OR_DROP, None, None, None,
+                          0.0, O, None, st)
+    torch.cuda.synchronize()
+    assert st_ref.item() == 0 and st.item() == 0
+    assert_close_out(O.reshape(-1, d), f64(ref).reshape(-1, d), "noalloc vs bsa_forward")
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy()
+    for h in range(H):
+        hrp, hci = orc.head_csr(rp_h, ci_h, h, M, 1)
+        want, _ = orc.keep_or_drop_head(f64(q[0, h].cpu()), f64(k[0, h].cpu()),
+                                        f64(v[0, h].cpu()), hrp, hci, block, 1 / math.sqrt(d))
+        assert_close_out(O[0, h], want, f"noalloc block-64 head {h} vs oracle")
