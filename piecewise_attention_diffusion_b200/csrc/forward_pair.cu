@@ -106,14 +106,15 @@ __device__ __forceinline__ void item_tile(const Params& p, int item, int& bh, in
   }
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool KP>
 struct Cfg {
   static constexpr int QBPT = kBQ / BKV;          // query blocks per tile (1 or 2)
+  static constexpr int KT = KP ? 2 * BKV : BKV;   // keys per exact step
   static constexpr int QBYTES = kBQ * D * 2;
   static constexpr int SLOT = kBQ * D * 2;        // a slot holds up to 128 rows x D
   static constexpr int NSLOT = D == 128 ? 5 : 8;
   static constexpr int SMEM = kStreams * QBYTES + NSLOT * SLOT + 1024;
-  static constexpr int HALF_EX = BKV / 2;         // columns of a half of an exact tile
+  static constexpr int HALF_EX = KT / 2;          // columns of a half of an exact tile
   static constexpr int HALF_D = D / 2;            // columns of a half of O
   __host__ __device__ static constexpr uint32_t S_COL(int x) { return 128u * x; }
   __host__ __device__ static constexpr uint32_t O_COL(int x) { return 256u + D * x; }
@@ -133,22 +134,56 @@ __device__ __forceinline__ int stream_item(int k, int x) {
   return blockIdx.x + (2 * k + x) * gridDim.x;
 }
 
+// The exact steps of a tile. Without KP a step is one key block j of its lists (merged);
+// with KP (64-token blocks, paired) a step is a pair m of key blocks 2m and 2m + 1, taken
+// once if the lists hold either, so that every step is a 128-key tile: the two softmax
+// halves of a row each own one block, and a row skips a half whose block is not in its
+// own list.
+template <bool KP>
+struct Steps {
+  Lists l;
+  int pend;  // with KP: the lists' next key block (-1 at the end)
+  __device__ __forceinline__ void init(const Lists& x) {
+    l = x;
+    if (KP) pend = l.next();
+  }
+  __device__ __forceinline__ int next() {
+    if (!KP) return l.next();
+    if (pend < 0) return -1;
+    const int m = pend >> 1;
+    pend = l.next();
+    if (pend >= 0 && (pend >> 1) == m) pend = l.next();
+    return m;
+  }
+};
+
+template <bool KP, int QBPT>
+__device__ __forceinline__ int count_steps(const Lists& l) {
+  if (!KP) return count_exact<QBPT>(l);
+  Steps<true> st;
+  st.init(l);
+  int n = 0;
+  while (st.next() >= 0) ++n;
+  return n;
+}
+
 // Per-stream position in the step schedule shared by the producer and the MMA issuer.
 // Steps of an item with n tiles: step 0 = S(0); step t (1 <= t < n) = PV(t-1), S(t);
 // step n = PV(n-1) [+ T] and the end of the item. An item with n = 0 has one step.
-template <int QBPT>
+template <int QBPT, bool KP>
 struct StreamPos {
   int k, item, bh, qt, n, n_ex, t;
   uint32_t tiles;  // tiles of earlier items of this stream (barrier phases)
   int items;       // earlier items of this stream
-  Lists lk, lv;    // K-side and V-side list cursors (producer)
+  Steps<KP> lk, lv;  // K-side and V-side step cursors (producer)
   __device__ __forceinline__ void start(const Params& p, int x, int n_ch) {
     item = stream_item(k, x);
     if (item >= p.n_items) return;
     item_tile(p, item, bh, qt);
-    lk = item_lists<QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
+    const Lists li = item_lists<QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
+    lk.init(li);
     lv = lk;
-    n_ex = count_exact<QBPT>(lk);
+    n_ex = count_steps<KP, QBPT>(li);
     n = n_ex + n_ch;
     t = 0;
   }
@@ -231,13 +266,13 @@ __device__ __forceinline__ float bf16_value(uint16_t u) {
   return __uint_as_float((uint32_t)u << 16);
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool KP>
 __global__ void __launch_bounds__(kThreads, 1)
 k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKb,
        const __grid_constant__ CUtensorMap tmVs, const __grid_constant__ CUtensorMap tmHb,
        const __grid_constant__ CUtensorMap tmO, const Params p) {
-  using C = Cfg<D, BKV>;
+  using C = Cfg<D, BKV, KP>;
   if (*p.flag) return;  // malformed lists: leave O untouched
 
   extern __shared__ unsigned char smem_raw[];
@@ -299,8 +334,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         unsigned char* dst = sSlot + slot * C::SLOT;
         const CUtensorMap* map = kind == kLoadK ? &tmK : kind == kLoadV ? &tmV
                                  : kind == kLoadKbar ? &tmKb : kind == kLoadVsum ? &tmVs : &tmHb;
-        const int rows = kind <= kLoadV ? BKV : (kind == kLoadHbar ? D : kChunk);
-        const int y = kind <= kLoadV ? j * BKV : (kind == kLoadHbar ? 0 : j * kChunk);
+        const int rows = kind <= kLoadV ? C::KT : (kind == kLoadHbar ? D : kChunk);
+        const int y = kind <= kLoadV ? j * C::KT : (kind == kLoadHbar ? 0 : j * kChunk);
         mbar_arrive_expect_tx(&bars.kv_full[slot], rows * D * 2);
         // one 4-D box: 64 columns x rows x (D/64) column groups; lands as D/64 swizzled
         // [rows x 64] sub-tiles, sub-tile h at byte offset h * rows * 128
@@ -309,7 +344,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         return true;
       };
       // the loads of one step of stream x, in the MMA issuer's order
-      auto step = [&](StreamPos<C::QBPT>& s, int x) -> bool {
+      auto step = [&](StreamPos<C::QBPT, KP>& s, int x) -> bool {
         if (s.t == 0) {
           if (s.n == 0) {
             s.advance(p, x, n_ch);
@@ -332,7 +367,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         s.advance(p, x, n_ch);
         return r;
       };
-      StreamPos<C::QBPT> s0, s1;
+      StreamPos<C::QBPT, KP> s0, s1;
       s0.k = s1.k = 0;
       s0.tiles = s1.tiles = 0;
       s0.items = s1.items = 0;
@@ -361,7 +396,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
       // of the most recent wait_slot
       uint32_t slot = 0, phase = 0, last = 0;
       bool ok = true;
-      constexpr uint32_t idesc_s_ex = idesc_bf16_f32(kBQ, BKV, false, false);
+      constexpr uint32_t idesc_s_ex = idesc_bf16_f32(kBQ, C::KT, false, false);
       constexpr uint32_t idesc_s_ch = idesc_bf16_f32(kBQ, kChunk, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, D, false, true);
       auto wait_slot = [&](uint32_t& addr) -> bool {
@@ -392,7 +427,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         }
       };
       // one step of stream x (see StreamPos); false when a wait gave up
-      auto mstep = [&](StreamPos<C::QBPT>& s, const int x) -> bool {
+      auto mstep = [&](StreamPos<C::QBPT, KP>& s, const int x) -> bool {
         if (s.t == 0) {
           // item start: its Q is loaded and the previous item's epilogue has read
           // this stream's S (first-order T) and O
@@ -409,7 +444,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
           uint32_t k_addr;
           if (!wait_slot(k_addr)) return false;
           const bool chunk = 0 >= s.n_ex;
-          issue_s(x, k_addr, chunk ? kChunk : BKV, chunk ? idesc_s_ch : idesc_s_ex);
+          issue_s(x, k_addr, chunk ? kChunk : C::KT, chunk ? idesc_s_ch : idesc_s_ex);
           release_slot();
           mma_commit(&bars.s_full[x]);
           s.t = 1;
@@ -426,7 +461,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         if (!mbar_wait(&bars.p_full[x], (s.tiles + u) & 1, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         {
-          const int kdim = u >= s.n_ex ? kChunk : BKV;
+          const int kdim = u >= s.n_ex ? kChunk : C::KT;
           const uint64_t b0 = smem_desc_sw128(v_addr, kdim * 128, 1024);
           // P of a kdim-key tile: half h (keys [h kdim/2, (h+1) kdim/2)) is packed at the
           // start of its own score columns, column h kdim/2 of the tile
@@ -439,7 +474,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         }
         if (more) {
           const bool chunk = s.t >= s.n_ex;
-          issue_s(x, k_addr, chunk ? kChunk : BKV, chunk ? idesc_s_ch : idesc_s_ex);
+          issue_s(x, k_addr, chunk ? kChunk : C::KT, chunk ? idesc_s_ch : idesc_s_ex);
           mma_commit(&bars.kv_empty[v_slot]);
           release_slot();
           mma_commit(&bars.s_full[x]);
@@ -464,7 +499,7 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
         s.advance(p, x, n_ch);
         return true;
       };
-      StreamPos<C::QBPT> s0, s1;
+      StreamPos<C::QBPT, KP> s0, s1;
       s0.k = s1.k = 0;
       s0.tiles = s1.tiles = 0;
       s0.items = s1.items = 0;
@@ -517,8 +552,10 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
       const int item = stream_item(k, x);
       int bh, qt;
       item_tile(p, item, bh, qt);
-      Lists lists = item_lists<C::QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
-      const int n_ex = count_exact<C::QBPT>(lists);
+      const Lists lists = item_lists<C::QBPT>(p.row_ptr, p.col_idx, p.csr_per_head, p.M, bh, qt);
+      Steps<KP> steps;
+      steps.init(lists);
+      const int n_ex = count_steps<KP, C::QBPT>(lists);
       const int n = n_ex + n_ch;
       const int row_g = qt * kBQ + row;
       const int iq = qt * C::QBPT + row / BKV;   // this row's query block
@@ -560,9 +597,19 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
           ex1 = __reduce_or_sync(kAll, w1) | t1;
           masked = true;
         } else {
-          int jt = -1;   // key block of the tile (needed for membership and padding)
-          if (C::QBPT == 2) {
-            jt = lists.next();
+          int jt = -1;   // key block of this half (needed for membership and padding)
+          if (C::QBPT == 2 && KP) {
+            // a pair of blocks: this row's own list may hold either; the half of the
+            // block it lacks is skipped
+            const int b0 = 2 * steps.next();
+            const bool in0 = mp < me && __ldg(p.col_idx + mp) == b0;
+            if (in0) ++mp;
+            const bool in1 = mp < me && __ldg(p.col_idx + mp) == b0 + 1;
+            if (in1) ++mp;
+            jt = b0 + hf;
+            skip = !(hf ? in1 : in0);
+          } else if (C::QBPT == 2) {
+            jt = steps.next();
             const bool member = mp < me && __ldg(p.col_idx + mp) == jt;
             if (member) ++mp;
             skip = !member;
@@ -572,7 +619,8 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
           // token padding: an exact tile of a block with fewer real tokens than its width
           // excludes its tail columns
           if (!skip && p.key_valid != nullptr && jt >= 0) {
-            const int v = min(max(__ldg(p.key_valid + jt), 1), BKV) - c0;
+            // (with KP the half is the whole block)
+            const int v = min(max(__ldg(p.key_valid + jt), 1), BKV) - (KP ? 0 : c0);
             if (v < w) {
               masked = true;
               tail_bits(v, ex0, ex1);
@@ -782,16 +830,16 @@ k_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensor
   }
 }
 
-template <int D, int BKV>
+template <int D, int BKV, bool KP>
 cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, const void* vs16,
                 const void* hb16, int Mp, cudaStream_t st) {
-  using C = Cfg<D, BKV>;
+  using C = Cfg<D, BKV, KP>;
   const Shape& s = a.s;
   const int BH = s.BH(), M = s.M();
   CUtensorMap tmQ, tmK, tmV, tmKb, tmVs, tmHb, tmO;
   const int qbox = s.L < kBQ ? s.L : kBQ;
   bool ok = make_map(&tmQ, a.Q, D, s.L, BH, qbox, qbox == kBQ) &&
-            make_map(&tmK, a.K, D, s.L, BH, BKV) && make_map(&tmV, a.V, D, s.L, BH, BKV);
+            make_map(&tmK, a.K, D, s.L, BH, C::KT) && make_map(&tmV, a.V, D, s.L, BH, C::KT);
   // the output map (128-row boxes) is used only when every query tile is 128 rows
   if (qbox == kBQ) ok = ok && make_map(&tmO, a.O, D, s.L, BH, kBQ);
   else tmO = tmQ;
@@ -823,11 +871,11 @@ cudaError_t run(const ForwardArgs& a, const int32_t* flag, const void* kb16, con
   p.flag = flag;
   p.status = a.status;
   p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitTimeoutNs;
-  cudaError_t e = cudaFuncSetAttribute(k_pair<D, BKV>,
+  cudaError_t e = cudaFuncSetAttribute(k_pair<D, BKV, KP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = min(p.n_items, sm_count());
-  k_pair<D, BKV><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, tmO, p);
+  k_pair<D, BKV, KP><<<grid, kThreads, C::SMEM, st>>>(tmQ, tmK, tmV, tmKb, tmVs, tmHb, tmO, p);
   return cudaGetLastError();
 }
 
@@ -838,8 +886,11 @@ cudaError_t launch_forward_pair(const ForwardArgs& a, const int32_t* flag, const
   // instantiated for head dim 64 only, the shape it is dispatched for
   const Shape& s = a.s;
   if (s.d != 64) return cudaErrorInvalidValue;
-  if (s.block == 64) return fwdpair::run<64, 64>(a, flag, kb16, vs16, hb16, Mp, st);
-  return fwdpair::run<64, 128>(a, flag, kb16, vs16, hb16, Mp, st);
+  // 64-token blocks go two to a 128-key step once the sequence holds a whole step (a
+  // K/V box of 128 rows must fit in the tensor)
+  if (s.block == 64 && s.L >= fwdpair::kBQ) return fwdpair::run<64, 64, true>(a, flag, kb16, vs16, hb16, Mp, st);
+  if (s.block == 64) return fwdpair::run<64, 64, false>(a, flag, kb16, vs16, hb16, Mp, st);
+  return fwdpair::run<64, 128, false>(a, flag, kb16, vs16, hb16, Mp, st);
 }
 
 }  // namespace bsa
