@@ -223,6 +223,11 @@ def test_forward_tiny_random_lists(mode):
     _forward_check(w, q, k, v, rp, ci, 1, mode, (kbar, vsum, Hbar))
 
 
+# (batch, head) slices of the multimodal workloads (8 x 16) compared with the oracle: one in
+# eight, spread over every batch, plus the last
+MULTIMODAL_SAMPLE = list(range(0, 128, 9)) + [127]
+
+
 @pytest.mark.parametrize("name", ["multimodal_dit", "multimodal_dit_padded"])
 def test_forward_multimodal_fixed_mask_keep_or_drop(name):
     """Without and with the token mask: in the padded workload the 77 text tokens fill
@@ -233,7 +238,7 @@ def test_forward_multimodal_fixed_mask_keep_or_drop(name):
     keep = orc.mask_dense(**w.mask)
     rp, ci = orc.dense_to_csr(keep)
     _forward_check(w, q, k, v, rp, ci, 0, b.MODE_KEEP_OR_DROP, None,
-                   heads_idx=[0, 17, 63, 127], key_valid=w.valid_tokens())
+                   heads_idx=MULTIMODAL_SAMPLE, key_valid=w.valid_tokens())
 
 
 @pytest.mark.parametrize("name", ["multimodal_pisa", "multimodal_pisa_padded"])
@@ -245,7 +250,7 @@ def test_forward_pisa_over_the_multimodal_fixed_mask(name):
     q, k, v = synth.make_qkv(w)
     keep = orc.mask_dense(**w.mask)
     rp, ci = orc.dense_to_csr(keep)
-    heads = [0, 17, 63, 127]
+    heads = MULTIMODAL_SAMPLE
     BH = w.batch * w.heads
     kf = f64(k).reshape(BH, w.seq_len, w.head_dim)
     vf = f64(v).reshape(BH, w.seq_len, w.head_dim)
@@ -429,7 +434,7 @@ def test_forward_list_checks_cross_the_32_entry_chunks():
 # --------------------------------------------------------- full workloads (sampled)
 @pytest.mark.parametrize("name,heads,qblocks", [
     ("image_pisa", [0, 13], None),
-    ("video_pisa", [0, 39], [0, 1, 63, 127]),
+    ("video_pisa", [0, 13, 26, 39], [0, 1, 31, 63, 64, 95, 126, 127]),
     ("text_image_pisa", [0, 11, 23], None),
 ])
 def test_pipeline_full_size_sampled(name, heads, qblocks):
