@@ -57,14 +57,18 @@ def test_selftest_rejects_bad_arguments():
         b.bsa_selftest_wait_timeout(20_000_000_000, st)
 
 
+@pytest.mark.parametrize("d,block", [(128, 128), (64, 64)])
 @pytest.mark.parametrize("mode", [b.MODE_KEEP_OR_DROP, b.MODE_PISA])
-def test_forward_abort_path_drains_frees_tmem_and_reports_timeout(mode):
+def test_forward_abort_path_drains_frees_tmem_and_reports_timeout(mode, d, block):
     """The attention kernel itself, with every bounded wait limited to a few ns: a wait
     runs out while TMA copies and MMAs are in flight, and the kernel's own abort path runs
     (abort flag, producer drains its copies, the MMA thread waits for its issued MMAs, TMEM
     freed). The call reports BSA_ERR_TIMEOUT; then, on the same context, the normal
-    forward matches the oracle. Limits of 1 us and 20 us end the same way or complete."""
-    w = synth.Workload("abort", 1, 8, 8192, 128, 128, "pisa", k_top=64, generator="iid")
+    forward matches the oracle. Limits of 1 us and 20 us end the same way or complete.
+    Head dim 128 runs the single-warpgroup kernel; head dim 64 (blocks of 64, two to a
+    step) the kernel whose row softmax is split between two warpgroups, which agree on
+    leaving through their named barrier."""
+    w = synth.Workload("abort", 1, 8, 8192, d, block, "pisa", k_top=64, generator="iid")
     q, k, v = synth.make_qkv(w, seed=21)
     BH, M = w.batch * w.heads, w.n_blocks
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -86,7 +90,7 @@ def test_forward_abort_path_drains_frees_tmem_and_reports_timeout(mode):
         torch.cuda.synchronize()
         elapsed = time.perf_counter() - t0
         code = st.item()
-        print(f"[abort] mode={mode} wait_ns={wait_ns} status={b.status_string(code)} "
+        print(f"[abort] mode={mode} d={d} wait_ns={wait_ns} status={b.status_string(code)} "
               f"{elapsed * 1e3:.2f} ms")
         assert elapsed < 5.0
         if wait_ns == 1:
