@@ -14,7 +14,9 @@
 // Two passes over K and V, because M_j needs H-bar, i.e. every block of the head:
 //   stats pass  writes kbar, vsum and, per head segment of its range, the partial sum
 //               of H_j (rows kept in registers; written once per segment);
-//   (a reduce kernel then forms H-bar from the partials in a fixed order);
+//   (a reduce kernel then forms H-bar from the partials in a fixed order; the norm pass
+//   is launched as its programmatic dependent, so that the norm pass's K/V stream starts
+//   while H-bar is formed, and only its epilogue waits for the reduce);
 //   norm pass   recomputes H_j and reduces ||H_j - H-bar||_F over the 128 rows.
 // Each pass is one persistent kernel; the flattened (head, block) range is dealt in
 // contiguous pieces of equal length, one per CTA (so every SM works, and a CTA meets
@@ -253,6 +255,9 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 #pragma unroll
     for (int c = 0; c < D; ++c) acc[c] = 0.f;
     int hb_head = -1;
+    // norm pass: H-bar comes from the reduce kernel, which this grid may overlap
+    // (programmatic dependent launch): wait for it to complete before the first read
+    if (!kStats) asm volatile("griddepcontrol.wait;" ::: "memory");
     BlockIter it;
     it.init(p);
     uint32_t n = 0;
@@ -376,6 +381,9 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 // ((bh + 1) M - 1) / per, and CTA c wrote its segment of head bh into slot c + bh.
 __global__ void k_reduce(const float* __restrict__ partial, int per, int grid, int M,
                          float* __restrict__ Hbar) {
+  // the norm pass may start now (programmatic dependent launch): its TMA and MMA warps
+  // read only K and V, and its epilogue waits for this grid before it reads H-bar
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int bh = blockIdx.y;
   if (e >= D * D) return;
@@ -464,8 +472,19 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
                                                                  Hbar);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.stats = false;
-  k_precompute<B, false><<<grid, kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
-  return cudaGetLastError();
+  // launched as a programmatic dependent of the reduce kernel, so that its K/V stream
+  // starts while H-bar is being formed
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cf::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_precompute<B, false>, tmK, tmV, p);
 }
 
 }  // namespace pretc
