@@ -11,7 +11,8 @@
 // malformed list sets BSA_ERR_BAD_CSR and the attention kernel leaves O untouched; with
 // token padding, a real-token count outside 1..block or, in the PISA modes, a list that
 // lacks a padded block sets BSA_ERR_BAD_PADDING the same way), then the tensor-core
-// attention kernel of forward_tc.cu.
+// attention kernel (forward_tc.cu dispatches by mode and head dim: forward_tc.cu for
+// head dim 128 and the per-block mode, forward_pair.cu for head dim 64).
 #include <math.h>
 
 #include "common.cuh"

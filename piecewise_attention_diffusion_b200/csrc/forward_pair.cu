@@ -42,7 +42,10 @@
 //           the freed score tile.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
 // Query tiles are 128 rows: one query block of 128, or two of 64 whose key-block lists
-// are merged (each row masks the key blocks its own block does not select).
+// are merged (each row masks the key blocks its own block does not select). With
+// 64-token blocks (and L >= 128) the exact steps are pairs of key blocks, 128 keys wide:
+// each half of a row owns one block of the pair and skips it when the row's own list
+// lacks it (see Steps).
 // Every mbarrier wait is bounded (sm100::mbar_wait); on a timeout the CTA drains its
 // in-flight copies and MMAs, frees TMEM and reports BSA_ERR_TIMEOUT.
 #include <limits.h>

@@ -1,4 +1,8 @@
-// bsa_forward on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+// bsa_forward on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), sm_100a: the
+// kernel for head dim 128 in the keep-or-drop and PISA modes, and for every head dim in
+// the per-block first-order mode (head dim 64 in the other two modes runs the kernel of
+// forward_pair.cu). This file also holds the launch dispatch and the statistics
+// conversion to bf16.
 //
 // Method ("多模态 DiT 上的块稀疏 Attention" §3.3/§4.4; "PISA: Piecewise Sparse Attention
 // Is Wiser for Efficient Diffusion Transformers", technical summary §2):
