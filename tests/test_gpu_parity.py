@@ -263,10 +263,14 @@ def test_forward_pisa_over_the_multimodal_fixed_mask(name):
 
 
 @pytest.mark.parametrize("L,block,d,kk", [(576, 64, 64, 3), (640, 128, 128, 2), (64, 64, 128, 1),
-                                          (128, 128, 128, 1), (64, 64, 64, 1),
-                                          (1152, 64, 128, 5), (768, 128, 64, 6)])
+                                          (128, 128, 128, 1), (64, 64, 64, 1), (128, 64, 64, 2),
+                                          (1088, 64, 64, 5), (1152, 64, 128, 5), (768, 128, 64, 6)])
 @pytest.mark.parametrize("mode", [b.MODE_KEEP_OR_DROP, b.MODE_PISA])
 def test_forward_shapes_and_ragged_tiles(L, block, d, kk, mode):
+    """Routed lists on small shapes of every (d, block) pair: one or two query blocks per
+    128-row tile, L below one tile, ragged last tiles. At d = 64, block 64 the kernel takes
+    key blocks two to a step once L >= 128: L = 128 is a single pair, and L = 576 and 1088
+    (an odd number of blocks) end with a pair whose second block lies past L."""
     w = synth.Workload("case", 1, 3, L, d, block, "pisa", k_top=kk, generator="block_centres")
     q, k, v = synth.make_qkv(w, seed=3)
     kbar, vsum, Hbar, Mn = _oracle_stats(k, v, block)
