@@ -182,14 +182,3 @@ def make_qkv(w: Workload, seed: int = 0, heads: list | None = None) -> tuple:
         return torch.stack(xs).reshape(shape).to(torch.bfloat16)
 
     return pack(qs), pack(ks), pack(vs)
-
-
-def random_csr(n_blocks: int, k_top: int, n_rows: int, seed: int = 0) -> tuple:
-    """Random sorted block lists with k_top entries per row (for parity tests)."""
-    g = torch.Generator().manual_seed(seed + 4242)
-    cols = []
-    for _ in range(n_rows):
-        cols.append(torch.sort(torch.randperm(n_blocks, generator=g)[:k_top]).values)
-    col_idx = torch.stack(cols).to(torch.int32).reshape(-1)
-    row_ptr = (torch.arange(n_rows + 1, dtype=torch.int32) * k_top)
-    return row_ptr, col_idx
