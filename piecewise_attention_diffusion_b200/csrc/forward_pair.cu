@@ -71,8 +71,9 @@ constexpr int kSoftmaxWarps = 4 * kStreams * kHalves;
 constexpr int kThreads = 32 * kSoftmaxWarps + 64;   // softmax warpgroups, producer, MMA issuer
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kProducerWarp + 1;
-// 576 threads, one CTA per SM: 112 registers per thread (65536 / 576, rounded down to a
-// multiple of 8), which holds a half score row (64 values) and its packed P.
+// 576 threads, one CTA per SM: 96 registers per thread. The register file is split over the
+// SM's four schedulers and two of them hold five of the 18 warps: 16384 / (5 * 32) rounded
+// down to a multiple of 8. That holds a half score row (64 values) and its packed P.
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kAll = 0xffffffffu;
