@@ -6,11 +6,12 @@ model and is not part of a PISA step). Default workload: video PISA, batch 1, 40
 L = 16384 (16 frames x 32 x 32), d = 128, block 128, density 12.5% (top-16 of 128).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu]
+                    [--workload NAME] [--shard replicas|heads] [--no-e2e] [--no-cpu]
 
 Prints ONE JSON line on rank 0. With torchrun (N > 1) every rank runs the same
-workload on its own GPU (replicas, weak scaling; the path needs no data exchange) and
-the time is the max over ranks.
+workload on its own GPU (replicas, weak scaling; the path needs no data exchange), or
+with --shard heads its own contiguous range of the workload's heads (strong scaling; the
+optional all-gather of O is timed apart from the step). The time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -201,6 +202,37 @@ def replica_value(flops_per_rank: float, ms_slowest: float, world: int) -> float
     return world * flops_per_rank / (ms_slowest * 1e-3) / 1e12
 
 
+def sum_over_ranks(x: float, world: int) -> float:
+    """The sum of every rank's x, on every rank."""
+    if world == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_value(flops_this_rank: float, ms_slowest: float, world: int, shard: str) -> float:
+    """Whole-job TFLOP/s, timed by the slowest rank. Replicas: every rank ran the whole
+    workload (weak scaling). Head shards: the ranks' FLOPs add up to the workload's (strong
+    scaling)."""
+    if shard == "heads":
+        return sum_over_ranks(flops_this_rank, world) / (ms_slowest * 1e-3) / 1e12
+    return replica_value(flops_this_rank, ms_slowest, world)
+
+
+def shard_workload(w, world: int, rank: int):
+    """This rank's part of `w` under head sharding: the workload restricted to the rank's
+    contiguous range of flattened (batch * heads) indices (batch 1), and that range."""
+    import dataclasses
+    from piecewise_attention_diffusion_b200.shard import head_range
+    BH = w.batch * w.heads
+    if world > BH:
+        raise SystemExit(f"--shard heads: {world} ranks for {BH} heads")
+    h0, h1 = head_range(BH, world, rank)
+    return dataclasses.replace(w, batch=1, heads=h1 - h0), (h0, h1)
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -298,7 +330,7 @@ def needs_flush(w) -> bool:
     return input_bytes(w) < 2 * L2_BYTES
 
 
-def config_of(w, world: int) -> dict:
+def config_of(w, world: int, shard: str = "replicas") -> dict:
     """The workload as both arms name it (identical keys and values)."""
     k_top = 0 if w.mask else w.top_k()
     l2 = (f"inputs larger than L2 (Q+K+V = {input_bytes(w) / 1e6:.0f} MB)" if not needs_flush(w)
@@ -308,7 +340,7 @@ def config_of(w, world: int) -> dict:
             "k_top": None if w.mask else k_top, "lambda": LAMBDA,
             "lists": "fixed multimodal mask (shared)" if w.mask else "bsa_route top-k",
             "real_tokens_per_block": w.valid_tokens() if w.key_valid else None,
-            "parallelism": f"replicas x{world}", "l2": l2}
+            "parallelism": f"{shard} x{world}", "l2": l2}
 
 
 class Path:
@@ -443,7 +475,15 @@ def run_sweep(args, world, rank, local) -> dict:
 def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    q, k, v = synth.make_qkv(w, seed=args.seed + rank)
+    w_full, shard = w, args.shard
+    if shard == "heads":
+        # this rank's heads of the one workload (the same bytes the whole run would hold)
+        w, (h0, h1) = shard_workload(w_full, world, rank)
+        q, k, v = (x.unsqueeze(0) for x in synth.make_qkv(w_full, seed=args.seed,
+                                                          heads=range(h0, h1)))
+    else:
+        # replicas: every rank runs the whole workload on its own seed
+        q, k, v = synth.make_qkv(w, seed=args.seed + rank)
     path = Path(w, q, k, v, dev)
     BH, L, d = w.batch * w.heads, w.seq_len, w.head_dim
 
@@ -452,7 +492,7 @@ def run_ours(args, w, world, rank, local):
     m = path.measure(args.steps, args.warmup, world)
     clk.t0, clk.t1 = m["t0"], m["t1"]
     ms_step, fwd_ms, F_fwd, F_step = m["ms_step"], m["fwd_ms"], m["F_fwd"], m["F_step"]
-    value = replica_value(F_step, ms_step, world)
+    value = job_value(F_step, ms_step, world, shard)
     pk = peaks()
     achieved = F_fwd / (fwd_ms * 1e-3) / 1e12
 
@@ -531,21 +571,41 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         serial_ms = max_over_ranks(s_s.elapsed_time(s_e) / n_serial, world)
-        e2e = {"value": round(replica_value(F_step, e2e_ms, world), 3), "unit": "TFLOP/s",
+        e2e = {"value": round(job_value(F_step, e2e_ms, world, shard), 3), "unit": "TFLOP/s",
                "ms_per_step": round(e2e_ms, 4), "pipelined": True, "depth": 2,
                "serial_ms_per_step": round(serial_ms, 4),
-               "serial_value": round(replica_value(F_step, serial_ms, world), 3),
+               "serial_value": round(job_value(F_step, serial_ms, world, shard), 3),
                "h2d_bytes_per_step": int(3 * q.numel() * 2),
                "d2h_bytes_per_step": int(O.numel() * 2)}
+
+    # head shards: the optional collective, an all-gather of O onto every rank, timed on
+    # its own after the steps (the path itself exchanges nothing)
+    o_gather = None
+    if shard == "heads" and world > 1:
+        from piecewise_attention_diffusion_b200.shard import gather_heads
+        n_all = w_full.batch * w_full.heads
+        full = gather_heads(path.O, n_all, world, rank)
+        torch.cuda.synchronize()
+        barrier(world)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(path.stream)
+        for _ in range(5):
+            full = gather_heads(path.O, n_all, world, rank)
+        g1.record(path.stream)
+        torch.cuda.synchronize()
+        o_gather = {"ms": round(max_over_ranks(g0.elapsed_time(g1) / 5, world), 4),
+                    "bytes_per_rank": int(full.numel() * full.element_size()),
+                    "in_step": False}
 
     clk.stop()
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if shard == "heads" else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: Q ~ N(0,1); K, V: " + GENERATOR_TEXT[w.generator] + ")",
-        "config": config_of(w, world),
+        "config": config_of(w_full, world, shard),
         "forward_ms": round(fwd_ms, 4), "forward_tflops": round(achieved, 3),
         "precompute_ms": round(m["pre_ms"], 4), "route_ms": round(m["route_ms"], 4),
         "forward_gflop": round(F_fwd / 1e9, 3),
@@ -561,6 +621,8 @@ def run_ours(args, w, world, rank, local):
     }
     if e2e:
         line["e2e"] = e2e
+    if o_gather:
+        line["o_gather"] = o_gather
     del path
     if not args.no_sweep:
         line["sweep"] = run_sweep(args, world, rank, local)
@@ -598,9 +660,10 @@ def run_reference(args, w, world, rank):
            "sample": info["sample"]}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (same generator and seed)",
-            "config": config_of(w, world),
+            "config": config_of(w, world, args.shard),
             "cpu_baseline": cpu,
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -616,6 +679,9 @@ def main():
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller profiling captures)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: every rank runs the whole workload (replicas, weak scaling) "
+                         "or its own range of the heads (strong scaling)")
     ap.add_argument("--cpu-heads", type=int, default=8)
     ap.add_argument("--ref-heads", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
