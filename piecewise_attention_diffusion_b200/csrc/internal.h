@@ -66,12 +66,6 @@ float forward_scale(float scale, int d);
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t st);
 
-// Tensor-core per-block statistics for d = 128 (precompute_tc.cu).
-size_t precompute_tc_workspace(const Shape& s);
-cudaError_t launch_precompute_tc(const Shape& s, const void* K, const void* V, float* kbar,
-                                 float* vsum, float* Hbar, float* Mnorm, float* Hblk, void* ws,
-                                 int32_t* status, cudaStream_t st);
-
 // Tensor-core attention kernel (forward_tc.cu); `flag` is the validation result, the
 // first word of the forward workspace.
 size_t forward_tc_workspace(const Shape& s);

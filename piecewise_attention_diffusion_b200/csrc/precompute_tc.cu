@@ -1,4 +1,4 @@
-// bsa_precompute for d = 128 on the tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+// bsa_precompute on the tensor cores (tcgen05 + TMEM + TMA), sm_100a, head dim 64 and 128.
 //
 // "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers",
 // technical summary §2: per KV block j the centroid kbar_j, the value sum vsum_j and
@@ -6,7 +6,10 @@
 // the H_j over the head and routing uses M_j = ||H_j - H-bar||.
 //
 // Per block the tensor core computes, from the K_j and V_j tiles exactly as TMA lands
-// them (both operands MN-major, 128-byte swizzled):
+// them (both operands MN-major, 128-byte swizzled; a head dimension of 64 is padded to
+// 128 in shared memory by a second 64-column sub-tile of zeros that TMA never writes, so
+// the products are the d = 128 ones with zero rows and columns past 64, and only the
+// real 64 x 64 corner is written out):
 //     C_j    = K_j^T V_j                  (d x d, fp32 in TMEM)
 //     ksum_j = K_j^T 1,  vsum_j = V_j^T 1  (against a tile of ones: exact column sums)
 // and the epilogue thread that owns row a of C applies the centring in fp32:
@@ -109,7 +112,7 @@ struct Barriers {
   uint64_t done;
 };
 
-template <int B, bool kStats>
+template <int B, int DO, bool kStats>
 __global__ void __launch_bounds__(kThreads, 1)
 k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
              const Params p) {
@@ -128,6 +131,13 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
   // ones tile (its swizzle is irrelevant: every element is 1.0)
   for (int e = threadIdx.x; e < C::ONES / 4; e += kThreads)
     reinterpret_cast<uint32_t*>(sOnes)[e] = 0x3F803F80u;  // bf16 pair (1.0, 1.0)
+  if constexpr (DO < D) {
+    // head dimension 64: the second 64-column sub-tile of every K and V tile stays zero
+    for (int t = 0; t < 2 * kStages; ++t) {
+      uint4* z = reinterpret_cast<uint4*>(smem + t * C::TILE + B * 128);
+      for (int e = threadIdx.x; e < B * 128 / 16; e += kThreads) z[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   if (threadIdx.x == 0) {
     abort_sh = 0;
     for (int i = 0; i < kStages; ++i) {
@@ -166,7 +176,7 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         const int st = n % kStages;
         if (!(ok = mbar_wait(&bars.empty[st], ((n / kStages) & 1) ^ 1, abort_flag))) break;
         unsigned char* dst = smem + st * C::STAGE;
-        mbar_arrive_expect_tx(&bars.full[st], C::STAGE);
+        mbar_arrive_expect_tx(&bars.full[st], 2u * B * DO * 2u);  // K and V, real columns
         tma_load_4d(dst, &tmK, &bars.full[st], 0, it.j * B, 0, it.bh);
         tma_load_4d(dst + C::TILE, &tmV, &bars.full[st], 0, it.j * B, 0, it.bh);
         ++n;
@@ -205,7 +215,7 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       if (p.key_valid != nullptr) {
         const int v = min(max(__ldg(p.key_valid + it.j), 1), B);
         if (v < B) {
-          constexpr int kChunks = (D / 64) * 8;  // 16-byte chunks of one row
+          constexpr int kChunks = (DO / 64) * 8;  // 16-byte chunks of one row's real columns
           for (int e = lane; e < 2 * (B - v) * kChunks; e += 32) {
             const int tile = e / ((B - v) * kChunks), rest = e % ((B - v) * kChunks);
             const int r = v + rest / kChunks, c = rest % kChunks;
@@ -251,9 +261,10 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int a = quad * 32 + lane;              // row of C = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     // stats: partial sum of H_j row a over the head segment; norm: H-bar row a of the head
-    float acc[D];
+    // (rows a >= DO of a padded head dimension are zero throughout and write nothing)
+    float acc[DO];
 #pragma unroll
-    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    for (int c = 0; c < DO; ++c) acc[c] = 0.f;
     int hb_head = -1;
     // norm pass: H-bar comes from the reduce kernel, which this grid may overlap
     // (programmatic dependent launch): wait for it to complete before the first read
@@ -267,14 +278,17 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       const uint32_t ph = (n >> 1) & 1;
       const int bh = it.bh, j = it.j;
       if (!kStats && bh != hb_head) {
-        const float4* src = reinterpret_cast<const float4*>(p.Hbar + ((size_t)bh * D + a) * D);
+        if (a < DO) {
+          const float4* src =
+              reinterpret_cast<const float4*>(p.Hbar + ((size_t)bh * DO + a) * DO);
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-          const float4 v = __ldg(src + c);
-          acc[4 * c] = v.x;
-          acc[4 * c + 1] = v.y;
-          acc[4 * c + 2] = v.z;
-          acc[4 * c + 3] = v.w;
+          for (int c = 0; c < DO / 4; ++c) {
+            const float4 v = __ldg(src + c);
+            acc[4 * c] = v.x;
+            acc[4 * c + 1] = v.y;
+            acc[4 * c + 2] = v.z;
+            acc[4 * c + 3] = v.w;
+          }
         }
         hb_head = bh;
       }
@@ -298,8 +312,8 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         kb = __uint_as_float(r0[0]) / (float)nv;
         vs = __uint_as_float(r1[0]);
       }
-      if (kStats) {
-        const size_t o = ((size_t)bh * p.M + j) * D + a;
+      if (kStats && a < DO) {
+        const size_t o = ((size_t)bh * p.M + j) * DO + a;
         p.kbar[o] = kb;
         p.vsum[o] = vs;
       }
@@ -310,9 +324,11 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       float sq = 0.f;
-      float* hrow = (!kStats && p.Hblk) ? p.Hblk + (((size_t)bh * p.M + j) * D + a) * D : nullptr;
+      float* hrow = (!kStats && p.Hblk && a < DO)
+                        ? p.Hblk + (((size_t)bh * p.M + j) * DO + a) * DO
+                        : nullptr;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < DO; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(base + c0, r);
         tmem_wait_ld();
@@ -356,10 +372,11 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         // (distinct per (CTA, head): the next CTA's first head is at least this one's
         // last) and start a new one
         float4* dst = reinterpret_cast<float4*>(
-            p.partial + (((size_t)blockIdx.x + bh) * D + a) * D);
+            p.partial + (((size_t)blockIdx.x + bh) * DO + a) * DO);
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-          dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+        for (int c = 0; c < DO / 4; ++c) {
+          if (a < DO)
+            dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
           acc[4 * c] = acc[4 * c + 1] = acc[4 * c + 2] = acc[4 * c + 3] = 0.f;
         }
       }
@@ -379,6 +396,7 @@ k_precompute(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
 // given grid: deterministic). CTA c covers blocks [c per, (c + 1) per) of the flattened
 // (head, block) range, so head bh's segments come from CTAs bh M / per ..
 // ((bh + 1) M - 1) / per, and CTA c wrote its segment of head bh into slot c + bh.
+template <int DO>
 __global__ void k_reduce(const float* __restrict__ partial, int per, int grid, int M,
                          float* __restrict__ Hbar) {
   // the norm pass may start now (programmatic dependent launch): its TMA and MMA warps
@@ -386,12 +404,12 @@ __global__ void k_reduce(const float* __restrict__ partial, int per, int grid, i
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int bh = blockIdx.y;
-  if (e >= D * D) return;
+  if (e >= DO * DO) return;
   const int c0 = (int)((int64_t)bh * M / per);
   const int c1 = min(grid - 1, (int)(((int64_t)bh * M + M - 1) / per));
   float s = 0.f;
-  for (int c = c0; c <= c1; ++c) s += partial[((size_t)c + bh) * D * D + e];
-  Hbar[(size_t)bh * D * D + e] = s / (float)M;
+  for (int c = c0; c <= c1; ++c) s += partial[((size_t)c + bh) * DO * DO + e];
+  Hbar[(size_t)bh * DO * DO + e] = s / (float)M;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -412,14 +430,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// K or V [BH][L][D] as 4-D (64 columns, L rows, D/64 groups, BH): one box = one block tile
-// landing as D/64 swizzled [B x 64] sub-tiles.
-bool make_map(CUtensorMap* m, const void* ptr, int L, int BH, int B) {
+// K or V [BH][L][d] as 4-D (64 columns, L rows, d/64 groups, BH): one box = one block tile
+// landing as d/64 swizzled [B x 64] sub-tiles.
+bool make_map(CUtensorMap* m, const void* ptr, int L, int BH, int B, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {64, (cuuint64_t)L, (cuuint64_t)(D / 64), (cuuint64_t)BH};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)D * L * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)B, (cuuint32_t)(D / 64), 1};
+  cuuint64_t dims[4] = {64, (cuuint64_t)L, (cuuint64_t)(d / 64), (cuuint64_t)BH};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, 128, (cuuint64_t)d * L * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)B, (cuuint32_t)(d / 64), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -434,19 +452,19 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int B>
+template <int B, int DO>
 cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float* vsum,
                 float* Hbar, float* Mnorm, float* Hblk, void* ws, int32_t* status,
                 cudaStream_t st) {
   using Cf = Cfg<B>;
   CUtensorMap tmK, tmV;
-  if (!make_map(&tmK, K, s.L, s.BH(), B) || !make_map(&tmV, V, s.L, s.BH(), B))
+  if (!make_map(&tmK, K, s.L, s.BH(), B, DO) || !make_map(&tmV, V, s.L, s.BH(), B, DO))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_precompute<B, true>,
+  cudaError_t e = cudaFuncSetAttribute(k_precompute<B, DO, true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_precompute<B, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Cf::SMEM);
+  e = cudaFuncSetAttribute(k_precompute<B, DO, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
   const int M = s.M(), sms = std::min(sm_count(), kMaxGrid);
   Params p;
@@ -466,10 +484,10 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   p.per_cta = ceil_div(p.n_units, sms);
   const int grid = ceil_div(p.n_units, p.per_cta);
   p.stats = true;
-  k_precompute<B, true><<<grid, kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
+  k_precompute<B, DO, true><<<grid, kThreads, Cf::SMEM, st>>>(tmK, tmV, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_reduce<<<dim3(ceil_div(D * D, 256), s.BH()), 256, 0, st>>>(p.partial, p.per_cta, grid, M,
-                                                                 Hbar);
+  k_reduce<DO><<<dim3(ceil_div(DO * DO, 256), s.BH()), 256, 0, st>>>(p.partial, p.per_cta,
+                                                                       grid, M, Hbar);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   p.stats = false;
   // launched as a programmatic dependent of the reduce kernel, so that its K/V stream
@@ -484,24 +502,29 @@ cudaError_t run(const Shape& s, const void* K, const void* V, float* kbar, float
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_precompute<B, false>, tmK, tmV, p);
+  return cudaLaunchKernelEx(&cfg, k_precompute<B, DO, false>, tmK, tmV, p);
 }
 
 }  // namespace pretc
 
-size_t precompute_tc_workspace(const Shape& s) {
+size_t precompute_workspace(const Shape& s) {
   // one partial sum per (CTA, head) segment: at most grid + BH - 1 slots, grid <= kMaxGrid
   // and <= the number of blocks
   const size_t grid = std::min<size_t>(pretc::kMaxGrid, (size_t)s.BH() * s.M());
-  return (grid + s.BH()) * pretc::D * pretc::D * sizeof(float);
+  return (grid + s.BH()) * (size_t)s.d * s.d * sizeof(float);
 }
 
-cudaError_t launch_precompute_tc(const Shape& s, const void* K, const void* V, float* kbar,
-                                 float* vsum, float* Hbar, float* Mnorm, float* Hblk, void* ws,
-                                 int32_t* status, cudaStream_t st) {
+cudaError_t launch_precompute(const Shape& s, const void* K, const void* V, float* kbar,
+                              float* vsum, float* Hbar, float* Mnorm, float* Hblk, void* ws,
+                              int32_t* status, cudaStream_t st) {
+  if (s.d == 64) {
+    if (s.block == 64)
+      return pretc::run<64, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+    return pretc::run<128, 64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+  }
   if (s.block == 64)
-    return pretc::run<64>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
-  return pretc::run<128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+    return pretc::run<64, 128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
+  return pretc::run<128, 128>(s, K, V, kbar, vsum, Hbar, Mnorm, Hblk, ws, status, st);
 }
 
 }  // namespace bsa

@@ -87,7 +87,7 @@ def _precompute_case(w, heads=None, seed=0):
 
 
 @pytest.mark.parametrize("name,heads", [("tiny_pisa", None), ("image_pisa", [0, 7, 23]),
-                                        ("video_pisa", [5])])
+                                        ("video_pisa", [5]), ("multimodal_pisa", [0, 77, 127])])
 def test_precompute_parity(name, heads):
     w = synth.workloads()[name]
     q, k, v = _precompute_case(w, heads)
