@@ -42,7 +42,7 @@ def _heads(x, heads):
     return x.reshape(BH, x.shape[2], x.shape[3])[heads]
 
 
-# d = 64 (mma.sync statistics kernel) and d = 128 (tcgen05 statistics kernel); the
+# d = 64 (the statistics kernel with its head dimension zero-padded to 128) and d = 128; the
 # second and the last case carry a one-token (timestep) block
 PRE_CASES = [
     ("multimodal_dit_padded", [0, 77, 127]),
