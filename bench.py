@@ -70,10 +70,10 @@ def needs_precompute(w) -> bool:
 
 def launches_per_step(w) -> int:
     """Kernels one step launches: precompute 3 (statistics, reduce, norm; skipped for a
-    fixed keep-or-drop mask), route 1 (not for a fixed mask), forward: list validation,
-    the PISA statistics' bf16 conversion, the forward kernel."""
+    fixed keep-or-drop mask), route 2 (pooling, scoring; not for a fixed mask), forward:
+    list validation, the PISA statistics' bf16 conversion, the forward kernel."""
     pre = 3 if needs_precompute(w) else 0
-    route = 0 if w.mask else 1
+    route = 0 if w.mask else 2
     fwd = 3 if w.mode == "pisa" else 2
     return pre + route + fwd
 

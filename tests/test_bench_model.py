@@ -36,9 +36,10 @@ def test_forward_bytes_closed_form():
 
 
 def test_launches_and_steps_per_workload():
-    # routed PISA: 3 precompute + 1 route + validation, statistics conversion, forward
-    assert bench.launches_per_step(W["video_pisa"]) == 7
-    assert bench.launches_per_step(W["sweep_L4096_d125_keep_or_drop"]) == 6
+    # routed PISA: 3 precompute + 2 route (pooling, scoring) + validation, statistics
+    # conversion, forward: the eight kernels of the step's ncu launch list
+    assert bench.launches_per_step(W["video_pisa"]) == 8
+    assert bench.launches_per_step(W["sweep_L4096_d125_keep_or_drop"]) == 7
     # a fixed keep-or-drop mask needs neither statistics nor routing
     assert not bench.needs_precompute(W["multimodal_dit"])
     assert bench.launches_per_step(W["multimodal_dit"]) == 2
