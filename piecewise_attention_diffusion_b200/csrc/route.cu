@@ -17,9 +17,11 @@
 //   k_route  one CTA per (head, 8 query blocks), one warp per query block:
 //     1. pooled query: the sum of the block's segment sums (workspace, L2) over its
 //        number of real rows;
-//     2. scores: eight lanes share a centroid row, so that every load of kbar (from L2)
+//     2. scores: eight lanes share a centroid row, so that every copy of kbar (from L2)
 //        reads whole 128-byte segments, and dot it with the CTA's 8 pooled queries in
-//        shared memory; a butterfly over the eight lanes adds the partial dots;
+//        shared memory; a butterfly over the eight lanes adds the partial dots. Each
+//        lane's chunks of the next pass's rows are copied (cp.async) into its own slots of
+//        shared memory while it computes this pass;
 //     3. softmax over the M blocks plus the normalised covariance term;
 //     4. exact top-k: the k-th largest score is found by a radix select on the float bit
 //        patterns (scores are >= 0, so the bit patterns order like the values), bit by
@@ -43,6 +45,10 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSeg = 32;                      // rows per pooling segment
 constexpr uint32_t kForcedKey = 0x7F800000u;  // bit pattern of +inf
+// shared-memory floats of the scoring pass's copy buffers: 2 passes x D/32 chunks of 16
+// bytes per thread
+template <int D>
+constexpr int kKvFloats = 2 * (D / 32) * kThreads * 4;
 
 // Column sums of every 32-row segment of Q over its real rows: partial[bh][seg][D].
 template <int B, int D>
@@ -102,23 +108,51 @@ k_pool(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ key_vali
 template <int D>
 __device__ __forceinline__ void score_block(const float* __restrict__ kb, bool vec, int M,
                                             float scale, const float* s_q, float* s_sc,
-                                            int warp, int lane) {
+                                            float4* s_kv, int warp, int lane) {
   constexpr int kG = 8;                 // lanes per centroid
   constexpr int kRows = 32 / kG;        // centroids per warp pass
   constexpr int kIt = D / (4 * kG);     // 16-byte chunks per lane per row
   static_assert(kWarps == kG, "lane g of a group writes query block g");
   const int g = lane % kG, rsub = lane / kG;
-  for (int j0 = warp * kRows; j0 < M; j0 += kWarps * kRows) {
-    const int j = j0 + rsub;
-    const bool valid = j < M;
-    const float* kr = kb + (size_t)(valid ? j : 0) * D;
-    float4 kv[kIt];
+  const int n_pass = (M - warp * kRows + kWarps * kRows - 1) / (kWarps * kRows);
+  // With 16-byte aligned rows, each lane copies its own chunks of the next pass's row into
+  // its private slots of shared memory (s_kv: 2 buffers x kIt per thread, thread-major),
+  // so that the copy overlaps this pass's arithmetic; it reads back only what it copied
+  // itself, which needs no barrier, only its own wait for the copy group.
+  auto copy_pass = [&](int ps) {
+    const int j = warp * kRows + ps * (kWarps * kRows) + rsub;
+    const float* kr = kb + (size_t)(j < M ? j : 0) * D;
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
-      const int c = (it * kG + g) * 4;
-      kv[it] = vec ? __ldg(reinterpret_cast<const float4*>(kr + c))
-                   : make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2),
-                                 __ldg(kr + c + 3));
+      const uint32_t dst = static_cast<uint32_t>(
+          __cvta_generic_to_shared(s_kv + ((ps & 1) * kIt + it) * kThreads + threadIdx.x));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                   "l"(kr + (it * kG + g) * 4)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (vec && n_pass > 0) copy_pass(0);
+  for (int ps = 0; ps < n_pass; ++ps) {
+    const int j = warp * kRows + ps * (kWarps * kRows) + rsub;
+    const bool valid = j < M;
+    float4 kv[kIt];
+    if (vec) {
+      if (ps + 1 < n_pass) {
+        copy_pass(ps + 1);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      }
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) kv[it] = s_kv[((ps & 1) * kIt + it) * kThreads + threadIdx.x];
+    } else {
+      const float* kr = kb + (size_t)(valid ? j : 0) * D;
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int c = (it * kG + g) * 4;
+        kv[it] = make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2), __ldg(kr + c + 3));
+      }
     }
     float acc[kWarps];
 #pragma unroll
@@ -166,7 +200,7 @@ __device__ __forceinline__ uint32_t select_kth(const uint32_t (&key)[NK], int k_
 // NK > 0: M <= 32 NK, and each lane keeps its scores (j = lane + 32 q) in registers from
 // the softmax to the compaction. NK == 0: any M, scores in shared memory.
 template <int B, int D, int NK>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)
 k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
         const float* __restrict__ Mnorm, const int32_t* __restrict__ key_valid, int L,
         int k_top, float lambda, float scale, int32_t* __restrict__ row_ptr,
@@ -178,7 +212,8 @@ k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
   const bool active = i < M;
 
   extern __shared__ __align__(16) float smem[];
-  float* s_q = smem;                            // kWarps x D (16-byte aligned rows)
+  float4* s_kv = reinterpret_cast<float4*>(smem);  // centroid chunks in flight, per thread
+  float* s_q = smem + kKvFloats<D>;             // kWarps x D (16-byte aligned rows)
   float* s_cov = s_q + kWarps * D;              // M
   float* s_sc = s_cov + M;                      // kWarps x M
   float* s_red = s_sc + kWarps * M;             // kWarps
@@ -221,7 +256,7 @@ k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
   //    loads when the caller's kbar allows them (each head's slice then does too, since
   //    M * D * 4 is a multiple of 16)
   const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
-  score_block<D>(kbar + (size_t)bh * M * D, vec, M, scale, s_q, s_sc, warp, lane);
+  score_block<D>(kbar + (size_t)bh * M * D, vec, M, scale, s_q, s_sc, s_kv, warp, lane);
   __syncthreads();
   if (!active) return;
 
@@ -373,10 +408,16 @@ cudaError_t run(const Shape& s, const void* Q, const float* kbar, const float* M
   k_pool<B, D><<<pool_grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), s.key_valid,
                                                s.L, n_seg, partial, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t sm = ((size_t)kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
+  const size_t sm =
+      ((size_t)kKvFloats<D> + kWarps * D + M + (size_t)kWarps * M + kWarps) * sizeof(float);
   const dim3 grid(ceil_div(M, kWarps), s.BH());
   auto go = [&](auto kern) -> cudaError_t {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (err != cudaSuccess) return err;
+    // five CTAs of the scoring kernel per SM (one wave at 40 heads of 128 blocks) need
+    // most of the SM's shared memory
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
     kern<<<grid, kThreads, sm, st>>>(partial, kbar, Mnorm, s.key_valid, s.L, k_top, lambda, scale,
                                      row_ptr, col_idx, scores, status);
