@@ -45,7 +45,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSeg = 32;                      // rows per pooling segment
 constexpr uint32_t kForcedKey = 0x7F800000u;  // bit pattern of +inf
-// shared-memory floats of the scoring pass's copy buffers: 2 passes x D/32 chunks of 16
+// shared-memory floats of the scoring pass's copy buffers: 2 buffers x D/32 chunks of 16
 // bytes per thread
 template <int D>
 constexpr int kKvFloats = 2 * (D / 32) * kThreads * 4;
@@ -252,9 +252,10 @@ k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
   const float cov = msum > 0.f ? lambda / msum : 0.f;
   for (int j = threadIdx.x; j < M; j += kThreads) s_cov[j] = cov * __ldg(mn + j);
 
-  // 2. block scores a_j = scale * qbar_w . kbar_j for the CTA's query blocks. 16-byte
-  //    loads when the caller's kbar allows them (each head's slice then does too, since
-  //    M * D * 4 is a multiple of 16)
+  // 2. block scores a_j = scale * qbar_w . kbar_j for the CTA's query blocks. The rows
+  //    are copied to shared memory 16 bytes at a time when the caller's kbar is 16-byte
+  //    aligned (each head's slice then is too, since M * D * 4 is a multiple of 16), and
+  //    read with scalar loads otherwise
   const bool vec = (reinterpret_cast<uintptr_t>(kbar) & 15u) == 0;
   score_block<D>(kbar + (size_t)bh * M * D, vec, M, scale, s_q, s_sc, s_kv, warp, lane);
   __syncthreads();
