@@ -19,8 +19,9 @@
 //        number of real rows;
 //     2. scores: eight lanes share a centroid row, so that every copy of kbar (from L2)
 //        reads whole 128-byte segments, and dot it with the CTA's 8 pooled queries in
-//        shared memory; a butterfly over the eight lanes adds the partial dots. Each
-//        lane's chunks of the next pass's rows are copied (cp.async) into its own slots of
+//        shared memory; each lane takes two rows, so that every pooled-query chunk it
+//        reads serves both; a butterfly over the eight lanes adds the partial dots. Each
+//        lane copies (cp.async) its chunks of the next pass's rows into its own slots of
 //        shared memory while it computes this pass;
 //     3. softmax over the M blocks plus the normalised covariance term;
 //     4. exact top-k: the k-th largest score is found by a radix select on the float bit
@@ -45,8 +46,8 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSeg = 32;                      // rows per pooling segment
 constexpr uint32_t kForcedKey = 0x7F800000u;  // bit pattern of +inf
-// shared-memory floats of the scoring pass's copy buffers: 2 buffers x D/32 chunks of 16
-// bytes per thread
+// shared-memory floats of the scoring pass's copy slots: D/32 chunks x 2 rows of 16 bytes
+// per thread
 template <int D>
 constexpr int kKvFloats = 2 * (D / 32) * kThreads * 4;
 
@@ -105,77 +106,109 @@ k_pool(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ key_vali
 // row, so each load instruction of a warp reads four rows in whole 128-byte segments; the
 // eight partial dots are added across the group by a butterfly, after which lane g holds
 // query w = g's score.
+// Wait until at most n of this thread's copy groups are pending (n a compile-time value).
+__device__ __forceinline__ void cp_async_wait(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+  }
+}
+
 template <int D>
 __device__ __forceinline__ void score_block(const float* __restrict__ kb, bool vec, int M,
                                             float scale, const float* s_q, float* s_sc,
                                             float4* s_kv, int warp, int lane) {
   constexpr int kG = 8;                 // lanes per centroid
-  constexpr int kRows = 32 / kG;        // centroids per warp pass
+  constexpr int kSub = 32 / kG;         // lane groups of a warp
+  constexpr int kRowsWarp = 2 * kSub;   // centroids per warp pass: two per lane
+  constexpr int kRowsCta = kWarps * kRowsWarp;
   constexpr int kIt = D / (4 * kG);     // 16-byte chunks per lane per row
   static_assert(kWarps == kG, "lane g of a group writes query block g");
+  static_assert(kIt <= 4, "copy-group waits");
   const int g = lane % kG, rsub = lane / kG;
-  const int n_pass = (M - warp * kRows + kWarps * kRows - 1) / (kWarps * kRows);
-  // With 16-byte aligned rows, each lane copies its own chunks of the next pass's row into
-  // its private slots of shared memory (s_kv: 2 buffers x kIt per thread, thread-major),
-  // so that the copy overlaps this pass's arithmetic; it reads back only what it copied
-  // itself, which needs no barrier, only its own wait for the copy group.
-  auto copy_pass = [&](int ps) {
-    const int j = warp * kRows + ps * (kWarps * kRows) + rsub;
-    const float* kr = kb + (size_t)(j < M ? j : 0) * D;
+  const int n_pass = (M - warp * kRowsWarp + kRowsCta - 1) / kRowsCta;
+  // Lane (g, rsub) takes rows rsub and rsub + kSub of each warp pass, so that every chunk
+  // of a pooled query read from shared memory serves two rows. With 16-byte aligned rows
+  // the chunks are copied (cp.async) into the thread's own slots of shared memory (s_kv:
+  // kIt chunks x 2 rows per thread, thread-major), one copy group per chunk: the next
+  // pass's chunk goes into the slots of this pass's chunk as soon as its arithmetic has
+  // consumed them. A thread reads back only what it copied itself: no barrier, only its
+  // own waits for its copy groups.
+  auto row_of = [&](int ps, int h) { return warp * kRowsWarp + ps * kRowsCta + rsub + h * kSub; };
+  auto copy_chunk = [&](int ps, int it) {
 #pragma unroll
-    for (int it = 0; it < kIt; ++it) {
+    for (int h = 0; h < 2; ++h) {
+      const int j = row_of(ps, h);
+      const float* kr = kb + (size_t)(j < M ? j : 0) * D;
       const uint32_t dst = static_cast<uint32_t>(
-          __cvta_generic_to_shared(s_kv + ((ps & 1) * kIt + it) * kThreads + threadIdx.x));
+          __cvta_generic_to_shared(s_kv + (it * 2 + h) * kThreads + threadIdx.x));
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
                    "l"(kr + (it * kG + g) * 4)
                    : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  if (vec && n_pass > 0) copy_pass(0);
+  if (vec && n_pass > 0) {
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) copy_chunk(0, it);
+  }
   for (int ps = 0; ps < n_pass; ++ps) {
-    const int j = warp * kRows + ps * (kWarps * kRows) + rsub;
-    const bool valid = j < M;
-    float4 kv[kIt];
-    if (vec) {
-      if (ps + 1 < n_pass) {
-        copy_pass(ps + 1);
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      }
+    const bool more = ps + 1 < n_pass;
+    float acc0[kWarps], acc1[kWarps];
 #pragma unroll
-      for (int it = 0; it < kIt; ++it) kv[it] = s_kv[((ps & 1) * kIt + it) * kThreads + threadIdx.x];
-    } else {
-      const float* kr = kb + (size_t)(valid ? j : 0) * D;
-#pragma unroll
-      for (int it = 0; it < kIt; ++it) {
-        const int c = (it * kG + g) * 4;
-        kv[it] = make_float4(__ldg(kr + c), __ldg(kr + c + 1), __ldg(kr + c + 2), __ldg(kr + c + 3));
-      }
-    }
-    float acc[kWarps];
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) acc[w] = 0.f;
+    for (int w = 0; w < kWarps; ++w) acc0[w] = acc1[w] = 0.f;
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
       const int c = (it * kG + g) * 4;
+      float4 k0, k1;
+      if (vec) {
+        // newer groups than this chunk's: this pass's later chunks, and (unless this is
+        // the last pass) the next pass's earlier chunks
+        cp_async_wait(more ? kIt - 1 : kIt - 1 - it);
+        k0 = s_kv[(it * 2) * kThreads + threadIdx.x];
+        k1 = s_kv[(it * 2 + 1) * kThreads + threadIdx.x];
+      } else {
+        const int j0 = row_of(ps, 0), j1 = row_of(ps, 1);
+        const float* r0 = kb + (size_t)(j0 < M ? j0 : 0) * D + c;
+        const float* r1 = kb + (size_t)(j1 < M ? j1 : 0) * D + c;
+        k0 = make_float4(__ldg(r0), __ldg(r0 + 1), __ldg(r0 + 2), __ldg(r0 + 3));
+        k1 = make_float4(__ldg(r1), __ldg(r1 + 1), __ldg(r1 + 2), __ldg(r1 + 3));
+      }
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
         const float4 qv = *reinterpret_cast<const float4*>(s_q + w * D + c);
-        acc[w] = fmaf(qv.w, kv[it].w,
-                      fmaf(qv.z, kv[it].z, fmaf(qv.y, kv[it].y, fmaf(qv.x, kv[it].x, acc[w]))));
+        acc0[w] = fmaf(qv.w, k0.w, fmaf(qv.z, k0.z, fmaf(qv.y, k0.y, fmaf(qv.x, k0.x, acc0[w]))));
+        acc1[w] = fmaf(qv.w, k1.w, fmaf(qv.z, k1.z, fmaf(qv.y, k1.y, fmaf(qv.x, k1.x, acc1[w]))));
+      }
+      // the slots of this chunk are consumed: refill them. The empty asm takes the loaded
+      // values as inputs, so the loads have completed before the copy is issued
+      if (vec && more) {
+        asm volatile("" ::"f"(k0.x), "f"(k0.y), "f"(k0.z), "f"(k0.w), "f"(k1.x), "f"(k1.y),
+                     "f"(k1.z), "f"(k1.w)
+                     : "memory");
+        copy_chunk(ps + 1, it);
       }
     }
 #pragma unroll
     for (int o = 1; o < kG; o <<= 1)
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) acc[w] += __shfl_xor_sync(0xffffffffu, acc[w], o);
-    float mine = acc[0];
+      for (int w = 0; w < kWarps; ++w) {
+        acc0[w] += __shfl_xor_sync(0xffffffffu, acc0[w], o);
+        acc1[w] += __shfl_xor_sync(0xffffffffu, acc1[w], o);
+      }
+    float mine0 = acc0[0], mine1 = acc1[0];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w)
-      if (g == w) mine = acc[w];
-    if (valid) s_sc[g * M + j] = scale * mine;
+    for (int w = 1; w < kWarps; ++w) {
+      if (g == w) {
+        mine0 = acc0[w];
+        mine1 = acc1[w];
+      }
+    }
+    const int j0 = row_of(ps, 0), j1 = row_of(ps, 1);
+    if (j0 < M) s_sc[g * M + j0] = scale * mine0;
+    if (j1 < M) s_sc[g * M + j1] = scale * mine1;
   }
 }
 
