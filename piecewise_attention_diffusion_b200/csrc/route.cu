@@ -24,9 +24,10 @@
 //        lane copies (cp.async) its chunks of the next pass's rows into its own slots of
 //        shared memory while it computes this pass;
 //     3. softmax over the M blocks plus the normalised covariance term;
-//     4. exact top-k: the k-th largest score is found by a radix select on the float bit
-//        patterns (scores are >= 0, so the bit patterns order like the values), bit by
-//        bit, with the keys in registers when M <= 256; ties at the threshold go to the
+//     4. exact top-k: a threshold of the k largest scores is found by a radix select on
+//        the float bit patterns (scores are >= 0, so the bit patterns order like the
+//        values), bit by bit until exactly k keys are at or above it, or to the last bit,
+//        with the keys in registers when M <= 256; ties at the threshold go to the
 //        smaller block index, and the selected indices are compacted in ascending order
 //        with ordered ballots.
 // Token padding: the pooled query of a block averages its real rows only, and every
@@ -212,10 +213,12 @@ __device__ __forceinline__ void score_block(const float* __restrict__ kb, bool v
   }
 }
 
-// The k-th largest of NK * 32 keys held in registers (key j = lane + 32 q; keys of absent
-// j are 0) by a bitwise radix select: from the top bit down, T keeps a bit when at least
-// k keys are >= T with it set. Bit 31 is the sign, 0 for every key. Every candidate has a
-// bit set, so keys of 0 are never counted.
+// The threshold of the k largest of NK * 32 keys held in registers (key j = lane + 32 q;
+// keys of absent j are 0) by a bitwise radix select: from the top bit down, T keeps a bit
+// when at least k keys are >= T with it set. Bit 31 is the sign, 0 for every key. Every
+// candidate has a bit set, so keys of 0 are never counted. The select stops as soon as
+// exactly k keys are >= T: they are then the k largest, whatever the lower bits (T is the
+// k-th largest key itself when it runs to the last bit).
 template <int NK>
 __device__ __forceinline__ uint32_t select_kth(const uint32_t (&key)[NK], int k_top) {
   uint32_t T = 0;
@@ -225,7 +228,10 @@ __device__ __forceinline__ uint32_t select_kth(const uint32_t (&key)[NK], int k_
 #pragma unroll
     for (int q = 0; q < NK; ++q) cnt += key[q] >= cand ? 1 : 0;
     cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= k_top) T = cand;
+    if (cnt >= k_top) {
+      T = cand;
+      if (cnt == k_top) break;
+    }
   }
   return T;
 }
@@ -340,14 +346,14 @@ k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
         if (key[q] == kForcedKey) key[q] = 0u;
     }
 
-    // 4. the k-th largest key, then 5. the ascending compaction: selected = key > T, or
-    //    key == T among the first ties_needed such keys in index order
+    // 4. the threshold of the k largest keys, then 5. the ascending compaction: selected =
+    //    key > T, or key == T among the first ties_needed such keys in index order
     const uint32_t T = select_kth<NK>(key, k_top);
     int greater = 0;
 #pragma unroll
     for (int q = 0; q < NK; ++q) greater += key[q] > T ? 1 : 0;
     greater = __reduce_add_sync(0xffffffffu, greater);
-    const int ties_needed = k_top - greater;  // >= 1
+    const int ties_needed = k_top - greater;  // >= 0
     int ties_seen = 0, out = 0;
 #pragma unroll
     for (int q = 0; q < NK; ++q) {
@@ -384,20 +390,24 @@ k_route(const float* __restrict__ partial, const float* __restrict__ kbar,
         if (__float_as_uint(scw[j]) == kForcedKey) scw[j] = 0.f;
     }
     __syncwarp();
-    // 4. k-th largest key by a bitwise radix select over shared memory: from the top bit
-    //    down, keep a bit of T when at least k keys are >= T with it set
+    // 4. the threshold of the k largest keys by a bitwise radix select over shared memory:
+    //    from the top bit down, keep a bit of T when at least k keys are >= T with it set,
+    //    and stop once exactly k keys are >= T
     uint32_t T = 0;
     for (int bit = 30; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
       int cnt = 0;
       for (int j = lane; j < M; j += 32) cnt += __float_as_uint(scw[j]) >= cand ? 1 : 0;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= k_top) T = cand;
+      if (cnt >= k_top) {
+        T = cand;
+        if (cnt == k_top) break;
+      }
     }
     int greater = 0;
     for (int j = lane; j < M; j += 32) greater += __float_as_uint(scw[j]) > T ? 1 : 0;
     greater = __reduce_add_sync(0xffffffffu, greater);
-    const int ties_needed = k_top - greater;  // >= 1
+    const int ties_needed = k_top - greater;  // >= 0
     // 5. ascending compaction
     int ties_seen = 0, out = 0;
     for (int j0 = 0; j0 < M; j0 += 32) {
